@@ -1,0 +1,31 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or
+execute this package: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it. It shares
+no code with the CUDA library and does not import it.
+
+Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
+
+- ``attention_forward``      standard three-step attention, full rows of S.
+  Pinned by: torch fp64 SDPA (library special case), closed forms (Q = 0,
+  N = 1, constant V), permutation equivariance/invariance, hand-worked golden
+  cases, and the blockwise online merge below.
+- ``attention_forward_rows`` the same for a chosen subset of query rows.
+  Pinned by: equality with the rows of ``attention_forward``.
+- ``attention_backward``     analytic gradients of the forward.
+  Pinned by: central finite differences on N <= 16, torch fp64 autograd.
+- ``blockwise_online_softmax_attention`` the tiled merge with running max and
+  running sum. Pinned by: equality with the full-row softmax on tiny inputs,
+  for several block sizes.
+
+No function here is "parity unpinned".
+"""
+
+from .attention import (  # noqa: F401
+    attention_forward,
+    attention_forward_rows,
+    attention_backward,
+    causal_visible,
+)
+from .online_softmax import blockwise_online_softmax_attention  # noqa: F401

@@ -1,0 +1,140 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+catch each one. A pin set that lets a dropped term, a wrong sign, an
+off-by-one mask or a transposed operand through would be no pin at all."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle.attention as att
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _golden_ok():
+    with open(GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        a = lambda x: np.asarray(x, dtype=np.float64)[None, None]  # noqa: E731
+        o, lse = att.attention_forward(a(c["q"]), a(c["k"]), a(c["v"]), c["scale"], c["causal"])
+        if not (np.allclose(o[0, 0], c["o"], rtol=0, atol=1e-12)
+                and np.allclose(lse[0, 0], c["lse"], rtol=0, atol=1e-12)):
+            return False
+        if "dq" in c:
+            g = att.attention_backward(a(c["q"]), a(c["k"]), a(c["v"]), a(c["do"]), c["scale"], c["causal"])
+            for name, t in zip(("dq", "dk", "dv"), g):
+                if not np.allclose(t[0, 0], c[name], rtol=0, atol=1e-12):
+                    return False
+    return True
+
+
+def _fd_ok(causal):
+    n, d, scale, h = 7, 3, 0.6, 1e-6
+    q, k, v, do = (_rand((1, 1, n, d), s) for s in (1, 2, 3, 4))
+
+    def loss(q_, k_, v_):
+        o, _ = att.attention_forward(q_, k_, v_, scale, causal)
+        return float(np.sum(o * do))
+
+    grads = att.attention_backward(q, k, v, do, scale, causal)
+    for which, g in enumerate(grads):
+        for idx in np.ndindex(*g.shape):
+            ap = [q.copy(), k.copy(), v.copy()]
+            am = [q.copy(), k.copy(), v.copy()]
+            ap[which][idx] += h
+            am[which][idx] -= h
+            num = (loss(*ap) - loss(*am)) / (2 * h)
+            if abs(num - g[idx]) > 1e-6 * max(1.0, abs(num)):
+                return False
+    return True
+
+
+def _closed_form_ok():
+    n = 9
+    q = np.zeros((1, 1, n, 2))
+    k, v = _rand((1, 1, n, 2), 5), _rand((1, 1, n, 2), 6)
+    _, lse = att.attention_forward(q, k, v, 1.0, True)
+    return np.allclose(lse[0, 0], np.log(np.arange(n) + 1), rtol=0, atol=1e-13)
+
+
+def test_unmutated_oracle_passes_all_checks():
+    assert _golden_ok() and _fd_ok(False) and _fd_ok(True) and _closed_form_ok()
+
+
+def test_mask_off_by_one_is_caught(monkeypatch):
+    monkeypatch.setattr(att, "causal_visible",
+                        lambda rows, n: np.arange(n)[None, :] <= np.asarray(rows)[:, None] - 1
+                        | (np.arange(n)[None, :] == 0))
+    assert not _closed_form_ok()
+
+
+def test_transposed_p_in_forward_is_caught(monkeypatch):
+    orig = att._forward_head
+
+    def bad(q, k, v, scale, causal, rows):
+        s = att._scores(q[rows], k, scale, rows, causal)
+        p, m, l = att._softmax_rows(s)
+        return p.T @ v, m + np.log(l)
+
+    monkeypatch.setattr(att, "_forward_head", bad)
+    assert not _golden_ok()
+    monkeypatch.setattr(att, "_forward_head", orig)
+
+
+def test_lse_missing_max_is_caught(monkeypatch):
+    def bad_softmax(s):
+        m = np.max(s, axis=1, keepdims=True)
+        e = np.exp(s - m)
+        l = np.sum(e, axis=1, keepdims=True)
+        return e / l, np.zeros(s.shape[0]), l[:, 0]
+
+    monkeypatch.setattr(att, "_softmax_rows", bad_softmax)
+    assert not _golden_ok()
+
+
+def _patch_backward(monkeypatch, variant):
+    def bwd(q, k, v, do, scale, causal):
+        N = q.shape[0]
+        r = np.arange(N)
+        s = att._scores(q, k, scale, r, causal)
+        p, _, _ = att._softmax_rows(s)
+        dp = do @ v.T
+        dd = np.sum(p * dp, axis=1, keepdims=True)
+        ds = p * (dp - dd)
+        dq, dk, dv = scale * (ds @ k), scale * (ds.T @ q), p.T @ do
+        if variant == "no_scale_dk":
+            dk = ds.T @ q
+        elif variant == "dropped_D":
+            dq = scale * ((p * dp) @ k)
+        elif variant == "sign":
+            dq = -dq
+        elif variant == "dv_untransposed":
+            dv = p @ do
+        elif variant == "D_rowsum_dp":
+            ds2 = p * (dp - np.sum(dp, axis=1, keepdims=True))
+            dq = scale * (ds2 @ k)
+        return dq, dk, dv
+
+    monkeypatch.setattr(att, "_backward_head", bwd)
+
+
+@pytest.mark.parametrize("variant", ["no_scale_dk", "dropped_D", "sign", "dv_untransposed", "D_rowsum_dp"])
+def test_backward_mistakes_are_caught(monkeypatch, variant):
+    _patch_backward(monkeypatch, "none")
+    assert _fd_ok(True) and _fd_ok(False)
+    _patch_backward(monkeypatch, variant)
+    assert not (_fd_ok(True) and _fd_ok(False))
+
+
+def test_scale_misapplied_is_caught(monkeypatch):
+    orig_scores = att._scores
+    monkeypatch.setattr(att, "_scores", lambda q, k, scale, rows, causal:
+                        orig_scores(q, k, math.sqrt(scale), rows, causal))
+    assert not _golden_ok()

@@ -1,0 +1,265 @@
+"""Pins for the fp64 oracle: facts fixed by the pages and by the mathematics,
+none of which re-types the oracle's own formula.
+
+- hand-worked closed-form cases (tests/golden/hand_cases.json);
+- the blockwise online-softmax merge of the pages equals the full-row softmax;
+- softmax rows sum to one and are invariant to a per-row shift of S;
+- constant V gives O equal to that constant;
+- closed forms for Q = 0 and N = 1;
+- permutation equivariance (Q rows) and invariance (joint K/V rows);
+- backward against central finite differences;
+- forward and backward against torch's fp64 CPU SDPA with autograd.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention_backward, attention_forward, attention_forward_rows
+from oracle import blockwise_online_softmax_attention
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def _rand(shape, seed, std=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * std
+
+
+def _as4(x):
+    return np.asarray(x, dtype=np.float64)[None, None]
+
+
+# ---------------------------------------------------------------- golden cases
+
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_golden_forward(case):
+    o, lse = attention_forward(_as4(case["q"]), _as4(case["k"]), _as4(case["v"]),
+                               case["scale"], case["causal"])
+    np.testing.assert_allclose(o[0, 0], np.array(case["o"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], np.array(case["lse"]), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("case", [c for c in _golden_cases() if "dq" in c], ids=lambda c: c["name"])
+def test_golden_backward(case):
+    dq, dk, dv = attention_backward(_as4(case["q"]), _as4(case["k"]), _as4(case["v"]),
+                                    _as4(case["do"]), case["scale"], case["causal"])
+    np.testing.assert_allclose(dq[0, 0], np.array(case["dq"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0], np.array(case["dk"]), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0], np.array(case["dv"]), rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------- blockwise merge == full rows
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("block", [1, 3, 64, 128, 256])
+@pytest.mark.parametrize("deferred", [True, False])
+def test_blockwise_online_merge_equals_full_rows(causal, block, deferred):
+    # Block sizes: 1 and 3 (ragged), 64 (pasted pseudocode, step 1),
+    # 128 and 256 (the V100 and A100 suggestions of cnnetsun.cn section 3.1).
+    n, d = 37, 8
+    q, k, v = _rand((n, d), 1), _rand((n, d), 2), _rand((n, d), 3)
+    scale = 1 / math.sqrt(d)
+    o_blk, lse_blk = blockwise_online_softmax_attention(q, k, v, scale, causal, block, deferred)
+    o, lse = attention_forward(q[None, None], k[None, None], v[None, None], scale, causal)
+    np.testing.assert_allclose(o_blk, o[0, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_blk, lse[0, 0], rtol=0, atol=1e-12)
+
+
+def test_blockwise_merge_large_logits():
+    # Logits of magnitude ~ 100 exercise the running-max correction.
+    n, d = 20, 4
+    q, k, v = _rand((n, d), 4, 10.0), _rand((n, d), 5, 10.0), _rand((n, d), 6)
+    o_blk, lse_blk = blockwise_online_softmax_attention(q, k, v, 1.0, True, 3, True)
+    o, lse = attention_forward(q[None, None], k[None, None], v[None, None], 1.0, True)
+    assert np.all(np.isfinite(o)) and np.max(np.abs(lse)) > 50
+    np.testing.assert_allclose(o_blk, o[0, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_blk, lse[0, 0], rtol=1e-14, atol=1e-12)
+
+
+# ------------------------------------------------------- softmax row properties
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_softmax_rows_sum_to_one(causal):
+    # With V = identity (N keys, N value dims) O is the probability matrix P.
+    n, d = 13, 5
+    q, k = _rand((1, 1, n, d), 7), _rand((1, 1, n, d), 8)
+    v = np.eye(n)[None, None]
+    p, _ = attention_forward(q, k, v, 0.7, causal)
+    p = p[0, 0]
+    assert np.all(p >= 0)
+    np.testing.assert_allclose(p.sum(axis=1), np.ones(n), rtol=0, atol=1e-14)
+    if causal:
+        assert np.all(p[np.triu_indices(n, 1)] == 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_row_shift_invariance(causal):
+    # Append a column c_i/scale to Q and a column of ones to K: S' = S + c_i.
+    # P (hence O) must not change; lse must shift by exactly c_i.
+    n, d, scale = 11, 6, 0.4
+    q, k, v = _rand((n, d), 9), _rand((n, d), 10), _rand((n, d), 11)
+    c = _rand((n,), 12, 5.0)
+    q2 = np.concatenate([q, (c / scale)[:, None]], axis=1)
+    k2 = np.concatenate([k, np.ones((n, 1))], axis=1)
+    o1, l1 = attention_forward(q[None, None], k[None, None], v[None, None], scale, causal)
+    o2, l2 = attention_forward(q2[None, None], k2[None, None], v[None, None], scale, causal)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2[0, 0], l1[0, 0] + c, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v(causal):
+    n, d = 17, 4
+    q, k = _rand((2, 3, n, d), 13), _rand((2, 3, n, d), 14)
+    row = np.array([1.5, -2.0, 0.25, 7.0])
+    v = np.broadcast_to(row, (2, 3, n, d)).copy()
+    o, _ = attention_forward(q, k, v, 0.5, causal)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-13)
+
+
+# ----------------------------------------------------------------- closed forms
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_closed_form(causal):
+    # Q = 0 makes every visible logit 0: uniform weights over visible keys.
+    n, d = 19, 3
+    q = np.zeros((1, 1, n, d))
+    k, v = _rand((1, 1, n, d), 15), _rand((1, 1, n, d), 16)
+    o, lse = attention_forward(q, k, v, 1.0, causal)
+    idx = np.arange(n)
+    if causal:
+        np.testing.assert_allclose(lse[0, 0], np.log(idx + 1), rtol=0, atol=1e-14)
+        prefix_mean = np.cumsum(v[0, 0], axis=0) / (idx + 1)[:, None]
+        np.testing.assert_allclose(o[0, 0], prefix_mean, rtol=0, atol=1e-13)
+    else:
+        np.testing.assert_allclose(lse[0, 0], np.full(n, math.log(n)), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(o[0, 0], np.broadcast_to(v[0, 0].mean(0), (n, d)), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_token(causal):
+    q, k, v = _rand((1, 2, 1, 8), 17), _rand((1, 2, 1, 8), 18), _rand((1, 2, 1, 8), 19)
+    o, lse = attention_forward(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, 0.3 * np.sum(q * k, axis=-1), rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------------ symmetries
+
+def test_query_permutation_equivariance():
+    n, d = 23, 5
+    q, k, v = _rand((1, 1, n, d), 20), _rand((1, 1, n, d), 21), _rand((1, 1, n, d), 22)
+    perm = np.random.default_rng(23).permutation(n)
+    o, lse = attention_forward(q, k, v, 0.5, False)
+    o_p, lse_p = attention_forward(q[:, :, perm], k, v, 0.5, False)
+    np.testing.assert_allclose(o_p, o[:, :, perm], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse_p, lse[:, :, perm], rtol=0, atol=1e-13)
+
+
+def test_joint_key_value_permutation_invariance():
+    n, d = 23, 5
+    q, k, v = _rand((1, 1, n, d), 24), _rand((1, 1, n, d), 25), _rand((1, 1, n, d), 26)
+    perm = np.random.default_rng(27).permutation(n)
+    o, lse = attention_forward(q, k, v, 0.5, False)
+    o_p, lse_p = attention_forward(q, k[:, :, perm], v[:, :, perm], 0.5, False)
+    np.testing.assert_allclose(o_p, o, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse_p, lse, rtol=0, atol=1e-13)
+
+
+def test_rows_subset_matches_full():
+    B, H, n, d = 2, 2, 300, 8
+    q, k, v = _rand((B, H, n, d), 28), _rand((B, H, n, d), 29), _rand((B, H, n, d), 30)
+    rows = np.array([0, 1, 127, 128, 255, 299])
+    heads = [(0, 1), (1, 0)]
+    for causal in (False, True):
+        o, lse = attention_forward(q, k, v, 0.35, causal)
+        o_r, lse_r = attention_forward_rows(q, k, v, 0.35, causal, heads, rows)
+        for t, (b, h) in enumerate(heads):
+            # same arithmetic, BLAS may block a row subset differently
+            np.testing.assert_allclose(o_r[t], o[b, h][rows], rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lse_r[t], lse[b, h][rows], rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------- finite differences
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 9, 16])
+def test_backward_central_finite_differences(causal, n):
+    d, scale, h = 4, 0.6, 1e-6
+    q, k, v, do = (_rand((1, 1, n, d), s) for s in (31, 32, 33, 34))
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward(q_, k_, v_, scale, causal)
+        return float(np.sum(o * do))
+
+    grads = attention_backward(q, k, v, do, scale, causal)
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.max(np.abs(num - g)) / max(1e-300, np.max(np.abs(g)))
+        if n == 1 and which in (0, 1):
+            # one token: O = V does not depend on q or k
+            assert np.max(np.abs(g)) == 0.0 and np.max(np.abs(num)) < 1e-9
+        else:
+            assert err <= 1e-6, (which, err)
+
+
+# ----------------------------------------------- library special case (torch)
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 8), (17, 16), (130, 64), (257, 32)])
+def test_against_torch_sdpa_fp64(causal, n, d):
+    B, H = 2, 3
+    q, k, v, do = (_rand((B, H, n, d), s) for s in (35, 36, 37, 38))
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+    to.backward(torch.tensor(do))
+    o, lse = attention_forward(q, k, v, scale, causal)
+    dq, dk, dv = attention_backward(q, k, v, do, scale, causal)
+    # Tolerance: assert_close(atol=1e-5, rtol=1e-3) of cnnetsun.cn section 5.2,
+    # tightened because both sides are fp64.
+    kw = dict(rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(o, to.detach().numpy(), **kw)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), **kw)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), **kw)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), **kw)
+    # lse via torch.logsumexp of the masked logits
+    s = torch.einsum("bhid,bhjd->bhij", torch.tensor(q), torch.tensor(k)) * scale
+    if causal:
+        s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), **kw)
+
+
+def test_backward_heads_subset_matches_full():
+    B, H, n, d = 1, 3, 40, 8
+    q, k, v, do = (_rand((B, H, n, d), s) for s in (39, 40, 41, 42))
+    full = attention_backward(q, k, v, do, 0.5, True)
+    sub = attention_backward(q, k, v, do, 0.5, True, heads=[(0, 2), (0, 0)])
+    for f, s in zip(full, sub):
+        np.testing.assert_allclose(s[0], f[0, 2], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(s[1], f[0, 0], rtol=0, atol=1e-13)
+
+
+def test_oracle_accepts_bf16_torch_inputs():
+    t = torch.randn(1, 1, 5, 4).to(torch.bfloat16)
+    o, _ = attention_forward(t, t, t, 0.5, True)
+    o2, _ = attention_forward(t.to(torch.float64).numpy(), t.to(torch.float64).numpy(),
+                              t.to(torch.float64).numpy(), 0.5, True)
+    np.testing.assert_array_equal(o, o2)
+    assert oracle.attention_forward is attention_forward
