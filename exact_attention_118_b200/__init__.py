@@ -1,0 +1,161 @@
+"""Python binding of libfa.so: exact, IO-aware fused attention for B200 (sm_100a).
+
+The functions ``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_size``,
+``fa_get_device_error``, ``fa_strerror`` and ``fa_version`` have the names and
+arguments of the C ABI in ``include/fa.h`` (pointers and the stream are plain
+integers) and only marshal arguments. ``attention_forward`` and
+``attention_backward`` are conveniences that take torch CUDA tensors, allocate
+the outputs with torch (device memory and streams are all torch supplies) and
+call the C ABI on the current stream. Every step of the computation runs in the
+library's CUDA kernels; there is no other path. If the library is missing the
+import of this package raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa.h")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_BF16, FA_F32 = 0, 1
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+_SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_get_device_error": (_I, [_P]),
+    "fa_strerror": (ctypes.c_char_p, [_I]),
+    "fa_version": (_I, []),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m exact_attention_118_b200.build` "
+            "(nvcc, sm_100a). There is no fallback path."
+        )
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def header_symbols():
+    """Names of the functions declared in include/fa.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:fa_status|size_t|const char\*|int)\s+(fa_\w+)\(", text, re.M)))
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {fa_strerror(status)} (status {status})")
+        self.status = status
+
+
+# ----------------------------------------------------------- C ABI, same names
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, o_dtype, stream) -> int:
+    return _lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, o_dtype, stream)
+
+
+def fa_bwd_workspace_size(B, H, N, d) -> int:
+    return _lib.fa_bwd_workspace_size(B, H, N, d)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, scale, causal, stream) -> int:
+    return _lib.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, scale, causal, stream)
+
+
+def fa_get_device_error(stream) -> int:
+    return _lib.fa_get_device_error(stream)
+
+
+def fa_strerror(status: int) -> str:
+    return _lib.fa_strerror(status).decode()
+
+
+def fa_version() -> int:
+    return _lib.fa_version()
+
+
+# ------------------------------------------------------ torch conveniences
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream_ptr(torch, device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def attention_forward(q, k, v, scale=None, causal=False, out_fp32=False, out=None, lse=None):
+    """O, lse = attention(q, k, v) on the GPU. q, k, v: contiguous bf16 CUDA
+    tensors [B, H, N, d]. Returns (O [B,H,N,d] bf16 or fp32, lse [B,H,N] fp32)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    if scale is None:
+        scale = d ** -0.5
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of equal shape")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, N, d,
+                float(scale), int(bool(causal)), FA_F32 if out.dtype == torch.float32 else FA_BF16,
+                _stream_ptr(torch, q.device))
+    _check(st, "fa_fwd")
+    return out, lse
+
+
+def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None):
+    """dQ, dK, dV of attention on the GPU, all bf16 [B, H, N, d]."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                B, H, N, d, float(scale), int(bool(causal)), _stream_ptr(torch, q.device))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def check_device_error(stream=None):
+    """Synchronise and raise FAError if a bounded device wait gave up."""
+    import torch
+
+    ptr = _stream_ptr(torch, None) if stream is None else stream
+    _check(fa_get_device_error(ptr), "device")

@@ -1,0 +1,370 @@
+// fa_fwd.cuh - fused attention forward for sm_100a (TMA + tcgen05 + TMEM).
+//
+// Method: "FlashAttention原理：从原始Attention到FlashAttention"
+// (blog.csdn.net/qq_43527718), sections 二.5-二.7, and "FlashAttention：优化大模型
+// 训练的内存与计算效率" (cnnetsun.cn), sections 2.1-2.2. Q is tiled against K/V
+// blocks held on chip; each block's scores are merged into the output with a
+// running row maximum m and running row sum l; O is divided by l once at the
+// end (the second FlashAttention's cut of non-matmul work, blog section 二.7);
+// query tiles form the outer loop and key/value tiles the inner loop (same
+// section); tiles wholly above the causal diagonal are never visited (same
+// section, third point). Only O and lse reach global memory.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and streams the
+// K/V tiles of that head through a shared-memory ring:
+//   warp 0      TMA producer: Q0, Q1 once; K_j, V_j into a KV_STAGES ring.
+//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM, then
+//               O_t += P_t V_j with P_t read from TMEM. The two tiles
+//               alternate so that the tensor core works on one tile while
+//               the other tile's softmax runs.
+//   warps 2-5   softmax warpgroup of tile 0 (one thread per query row).
+//   warps 6-9   softmax warpgroup of tile 1.
+// TMEM columns (512 allocated): S0/P0 [0,128), S1/P1 [128,256),
+// O0 [256, 256+D), O1 [256+D, 256+2D).
+//
+// Softmax per row, in log2 units (lambda = scale*log2(e)):
+//   m_blk = lambda * max_j S_ij;  if m_blk > m + 8 the running max moves to
+//   m_blk and O, l are multiplied by alpha = 2^(m_old - m_new) (else m stays:
+//   the result is the same because O and l share the same stale m, and the
+//   largest p is at most 2^8);  p_ij = 2^(lambda*S_ij - m);  l = alpha*l + sum p.
+//   Epilogue: O /= l;  lse = ln2 * (m + log2 l).
+#pragma once
+#include <cuda.h>
+#include "fa_ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int BH;
+  int N;
+  int n_pairs;       // ceil(N / 256): CTAs per (batch, head)
+  float scale_log2;  // scale * log2(e)
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTile = 128 * D * 2;          // one 128 x D bf16 tile
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTile;
+  static constexpr int kK = 2 * kTile;
+  static constexpr int kV = kK + kStages * kTile;
+  static constexpr int kBar = kV + kStages * kTile;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KB alignment
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+constexpr int kFwdThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D, bool CAUSAL, bool OF32>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  constexpr int S = L::kStages;
+  constexpr int KCH = D / 64;  // 64-column (128-byte) chunks per row
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;  // [2]
+  uint64_t* p_full = s_full + 2;   // [2]
+  uint64_t* o_full = p_full + 2;   // [2]
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+
+  // Causal: heaviest query tiles first across all heads. Otherwise head-major
+  // so CTAs that read the same K/V run together and share it through L2.
+  int pair, bh;
+  if (CAUSAL) {
+    pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / p.BH;
+    bh = static_cast<int>(blockIdx.x) % p.BH;
+  } else {
+    bh = static_cast<int>(blockIdx.x) / p.n_pairs;
+    pair = static_cast<int>(blockIdx.x) % p.n_pairs;
+  }
+  const int q0 = pair * 256;
+  const int n_kv = (N + 127) / 128;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qs = q0 + 128 * t;
+    n_t[t] = (qs >= N) ? 0 : (CAUSAL ? min(n_kv, qs / 128 + 1) : n_kv);
+  }
+  const int J = max(n_t[0], n_t[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, 128);
+      mbar_init(o_full + t, 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * 64, q0 + 128 * t, bh);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < J; ++j) {
+        const int s = j % S, u = j / S;
+        if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(k_full + s, L::kTile);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, j * 128, bh);
+        k_issued = j + 1;
+        if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(v_full + s, L::kTile);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, j * 128, bh);
+        v_issued = j + 1;
+      }
+      // Every copy this thread started must land before the CTA exits.
+      wait_parity_drain(q_full, 0);
+      for (int j = max(0, k_issued - S); j < k_issued; ++j) wait_parity_drain(k_full + j % S, (j / S) & 1);
+      for (int j = max(0, v_issued - S); j < v_issued; ++j) wait_parity_drain(v_full + j % S, (j / S) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);  // Q, K both K-major
+      constexpr uint32_t kIdO = idesc_bf16(128, D, 0, 1);    // P (TMEM), V MN-major
+      const uint32_t q_addr[2] = {smem_u32(smem + L::kQ0), smem_u32(smem + L::kQ1)};
+      const uint32_t k_addr = smem_u32(smem + L::kK);
+      const uint32_t v_addr = smem_u32(smem + L::kV);
+
+      auto issue_s = [&](int t, int stage) {
+        const uint32_t ka = k_addr + stage * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, sdesc_sw128(q_addr[t] + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdS,
+                 kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t va = v_addr + stage * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), kIdO,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = wait_parity(q_full, 0, abort_flag) && wait_parity(k_full, 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) {
+            issue_s(t, 0);
+            mma_commit(s_full + t);
+          }
+        mma_commit(k_empty + 0);
+      }
+      for (int j = 0; ok && j < J; ++j) {
+        const int s = j % S;
+        if (!(ok = wait_parity(v_full + s, (j / S) & 1, abort_flag))) break;
+        tc_fence_after();
+        const int jn = j + 1, sn = jn % S;
+        bool k_next = false;
+        for (int t = 0; t < 2; ++t) {
+          if (j < n_t[t]) {
+            if (!(ok = wait_parity(p_full + t, j & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_pv(t, s, j > 0);
+            mma_commit(o_full + t);
+          }
+          if (t == 1) mma_commit(v_empty + s);
+          if (jn < n_t[t]) {
+            if (!k_next) {
+              if (!(ok = wait_parity(k_full + sn, (jn / S) & 1, abort_flag))) break;
+              tc_fence_after();
+              k_next = true;
+            }
+            issue_s(t, sn);
+            mma_commit(s_full + t);
+          }
+        }
+        if (ok && jn < J) mma_commit(k_empty + sn);
+      }
+      // Let every MMA this thread issued finish before TMEM is freed.
+      mma_commit(mma_done);
+      wait_parity_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    const int qi = q0 + 128 * t + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const int nt = n_t[t];
+    const float lam = p.scale_log2;
+
+    float m = -INFINITY;  // running max, log2 units
+    float l = 0.f;        // running sum
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      ok = __all_sync(0xffffffffu, wait_parity(s_full + t, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t sr[128];
+        tmem_ld32(tS + 0, sr + 0);
+        tmem_ld32(tS + 32, sr + 32);
+        tmem_ld32(tS + 64, sr + 64);
+        tmem_ld32(tS + 96, sr + 96);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+      }
+      const int kb = j * 128;
+      if (kb + 128 > N || (CAUSAL && kb + 127 > q0 + 128 * t)) {
+        int lim = N - kb;
+        if (CAUSAL) lim = min(lim, qi - kb + 1);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * lam;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_blk > m + kRescaleThreshold) {
+        alpha = ex2(m - m_blk);  // 0 on the first visited block (m = -inf)
+        m = m_blk;
+        rescale = true;
+      }
+      const float neg_m = -m;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2(fmaf(s[2 * c], lam, neg_m));
+        const float p1 = ex2(fmaf(s[2 * c + 1], lam, neg_m));
+        rs0 += p0;
+        rs1 += p1;
+        pk[c] = pack_bf16(p0, p1);
+      }
+      l = l * alpha + (rs0 + rs1);
+      tmem_st32(tS + 0, pk + 0);
+      tmem_st32(tS + 32, pk + 32);
+      if (j > 0) {
+        // PV_{j-1} finished before S_j (same issuing thread, committed
+        // earlier), so this wait is immediate; it keeps the phase count exact.
+        ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        if (__any_sync(0xffffffffu, rescale)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + c, ov);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok && nt > 0) {
+      ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (nt - 1) & 1, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool valid = qi < N;
+        const size_t row = static_cast<size_t>(bh) * N + (valid ? qi : 0);
+        if (valid) p.lse[row] = (m + log2f(l)) * 0.69314718055994531f;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c, ov);
+          tmem_wait_ld();
+          if (valid) {
+            if (OF32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row * D + c);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l, __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                     __uint_as_float(ov[4 * e + 2]) * inv_l, __uint_as_float(ov[4 * e + 3]) * inv_l);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D + c);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint4 w;
+                w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                dst[e] = w;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,181 @@
+// fa_host.cu - the C ABI declared in include/fa.h: argument checks, TMA
+// descriptor encoding, launch configuration and status codes. The whole
+// library is this one translation unit (kernels come in through headers).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// The kernels use tcgen05 and TMA: compute capability 10.0 (sm_100a) only.
+fa_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_sizes(int B, int H, int N, int d, float scale, int causal) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// [BH][N][inner] row-major tensor viewed by TMA as dims {inner, N, BH}, with a
+// box of {box_inner, box_rows, 1}. Out-of-range rows of a head read as zero
+// and are clipped on store, so a ragged N never touches the next head.
+fa_status make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int inner, int N,
+                    int BH, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem_bytes,
+                                 static_cast<cuuint64_t>(inner) * elem_bytes * N};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, int d, int N, int BH) {
+  return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <typename Kern>
+fa_status launch_status(Kern) {
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool OF32>
+fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
+                     cudaStream_t st) {
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OF32>;
+  const int smem = fa::FwdLayout<D>::kAlloc;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
+  kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, p);
+  return launch_status(kern);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_strerror(fa_status s) {
+  switch (s) {
+    case FA_OK: return "success";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, fa_dtype o_dtype, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  fa_status s = check_sizes(B, H, N, d, scale, causal);
+  if (s != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const int BH = B * H;
+  alignas(64) CUtensorMap tq, tk, tv;
+  if ((s = make_bf16_tile_map(&tq, q, d, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tk, k, d, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tv, v, d, N, BH)) != FA_OK) return s;
+
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.BH = BH;
+  p.N = N;
+  p.n_pairs = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool f32 = (o_dtype == FA_F32);
+  if (d == 64) {
+    if (causal) return f32 ? launch_fwd<64, true, true>(tq, tk, tv, p, st) : launch_fwd<64, true, false>(tq, tk, tv, p, st);
+    return f32 ? launch_fwd<64, false, true>(tq, tk, tv, p, st) : launch_fwd<64, false, false>(tq, tk, tv, p, st);
+  }
+  if (causal) return f32 ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
+  return f32 ? launch_fwd<128, false, true>(tq, tk, tv, p, st) : launch_fwd<128, false, false>(tq, tk, tv, p, st);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d, 1.f, 0) != FA_OK) return 0;
+  return fa::bwd_workspace_bytes(B * H, N, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  fa_status s = check_sizes(B, H, N, d, scale, causal);
+  if (s != FA_OK) return s;
+  if (ws_bytes < fa::bwd_workspace_bytes(B * H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((s = check_device()) != FA_OK) return s;
+  return fa::bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, d, scale, causal,
+                        static_cast<cudaStream_t>(stream), make_bf16_tile_map, make_tmap);
+}
+
+fa_status fa_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0u;
+  if (cudaMemcpyFromSymbol(&word, fa::g_device_error, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0u) {
+    const unsigned int zero = 0u;
+    if (cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+/*
+ * fa.h - C ABI of a B200 (sm_100a) library of exact, IO-aware fused
+ * scaled-dot-product attention: forward and backward.
+ *
+ * What it computes. For each batch b and head h, with Q, K, V of size N x d
+ * ("FlashAttention原理：从原始Attention到FlashAttention", blog.csdn.net/qq_43527718,
+ * section 二.2, the standard computation):
+ *     S = scale * Q K^T,  P = softmax(S) row by row,  O = P V.
+ * The library never forms S or P in global memory: Q is tiled against K/V
+ * blocks held on chip and the row softmax is merged block by block with a
+ * running maximum and running sum (same page, sections 二.5 and 二.6;
+ * "FlashAttention：优化大模型训练的内存与计算效率", cnnetsun.cn, sections 2.1 and
+ * 2.2). Only O and the per-row log-sum-exp go back to global memory. The
+ * backward recomputes P tile by tile from that stored log-sum-exp instead of
+ * reading a stored N x N matrix (blog section 二, "做法", second strategy).
+ *
+ * Conventions shared by every call:
+ *   Layout     q, k, v, o, dO, dq, dk, dv are dense, contiguous [B, H, N, d]
+ *              row-major tensors (the [B, H, N, d] shape of the pasted
+ *              pseudocode on the blog page, step 1). lse is [B, H, N] fp32.
+ *   dtypes     q, k, v, dO, dq, dk, dv: bf16. o: bf16 or fp32 in fa_fwd
+ *              (o_dtype), bf16 in fa_bwd.
+ *   Pointers   device pointers (CUDA global memory of the current device),
+ *              each 16-byte aligned. The caller owns every buffer, including
+ *              the backward workspace. The library allocates no device memory;
+ *              it keeps only a small host-side cache of launch descriptors.
+ *   Sizes      B >= 1, H >= 1, N >= 1 (any value, ragged tails are handled),
+ *              d in {64, 128}, B*H*N < 2^31.
+ *   scale      the factor applied to Q K^T (1/sqrt(d) in the pages' pseudocode,
+ *              step 3); any finite value > 0.
+ *   causal     0: every key visible. 1: key j visible to query i iff j <= i
+ *              (the autoregressive mask named by is_causal in cnnetsun.cn
+ *              section 3.1); tiles entirely above the diagonal are skipped
+ *              (blog section 二.7, third point).
+ *   stream     a cudaStream_t passed as void*; NULL means the legacy default
+ *              stream. All work is asynchronous on that stream.
+ *   Errors     argument errors come back synchronously, before any launch,
+ *              as FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED. A failed launch
+ *              returns FA_ERR_CUDA. Every device-side wait in the kernels has
+ *              a time limit; if one gives up, the kernel records it in a
+ *              device error word and returns early, and fa_get_device_error
+ *              reports FA_ERR_TIMEOUT.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or scale */
+  FA_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. d = 96) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+
+/*
+ * Forward pass. Writes O (o_dtype) and lse = ln(sum_j exp(scale * q_i . k_j))
+ * over visible j, natural log, fp32 (the stored softmax normalisation factor
+ * of blog section 二 "做法"; log space per cnnetsun.cn section 2.2).
+ * Reads q, k, v once from global memory per CTA's tiles; writes O and lse once.
+ * Inputs: q, k, v (bf16 [B,H,N,d]). Outputs: o ([B,H,N,d], o_dtype), lse
+ * (fp32 [B,H,N]).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float scale, int causal, fa_dtype o_dtype,
+                 void* stream);
+
+/*
+ * Bytes of caller-owned device workspace fa_bwd needs: a fp32 [B,H,N,d]
+ * accumulator for dQ plus the fp32 [B,H,N] row-dot D = rowsum(dO * O),
+ * rounded up to 256-byte pieces. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass. Given the forward inputs, its outputs o (bf16) and lse, and
+ * the upstream gradient dO, writes dq, dk, dv (bf16 [B,H,N,d]):
+ *     dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO_i * O_i),
+ *     dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q,
+ * with P recomputed on chip from q, k and lse (blog section 二.5, second point).
+ * Launches, in order on `stream`: a memset of the dQ accumulator, the dO.O
+ * row-dot kernel, the main kernel (loops over query tiles for each key tile,
+ * accumulating dK and dV on chip and adding dQ contributions into the fp32
+ * accumulator), and a kernel that converts the accumulator to bf16 dq.
+ * workspace: device pointer, 256-byte aligned, at least
+ * fa_bwd_workspace_size(B,H,N,d) bytes (else FA_ERR_INVALID_ARG). Its
+ * contents on entry do not matter; on exit they are scratch.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                 int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word.
+ * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
+ * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.
+ */
+fa_status fa_get_device_error(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_strerror(fa_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/fa.h declares, and rejects bad arguments before it
+touches the device."""
+
+import ctypes
+
+import pytest
+
+import exact_attention_118_b200 as fa
+
+FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
+
+
+def test_library_loads_and_exports_every_header_symbol():
+    names = fa.header_symbols()
+    assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_error",
+                          "fa_strerror", "fa_version"}
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror_and_version():
+    assert fa.fa_strerror(fa.FA_OK) == "success"
+    for s in range(1, 5):
+        assert fa.fa_strerror(s) and fa.fa_strerror(s) != "success"
+    assert fa.fa_strerror(99) == "unknown status"
+    assert fa.fa_version() >= 100
+
+
+def test_workspace_size():
+    B, H, N, d = 2, 3, 1000, 128
+    rows = B * H * N
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert fa.fa_bwd_workspace_size(B, H, N, d) == up(rows * d * 4) + up(rows * 4)
+    assert fa.fa_bwd_workspace_size(0, 1, 1, 64) == 0
+    assert fa.fa_bwd_workspace_size(1, 1, 1, 96) == 0
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, N=16, d=64, scale=0.125, causal=0,
+             o_dtype=fa.FA_BF16, stream=None)
+    a.update(kw)
+    return fa.fa_fwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=FAKE + 4), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_ERR_INVALID_ARG),
+    (dict(B=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(H=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=7), fa.FA_ERR_INVALID_ARG),
+    (dict(B=1 << 16, H=1 << 10, N=1 << 10), fa.FA_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_arguments_without_launching(kw, want):
+    assert _fwd(**kw) == want
+
+
+def _bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dO=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE,
+             ws_bytes=1 << 30, B=1, H=1, N=16, d=64, scale=0.125, causal=1, stream=None)
+    a.update(kw)
+    return fa.fa_bwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(dO=None), fa.FA_ERR_INVALID_ARG),
+    (dict(dq=FAKE + 2), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=None), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16), fa.FA_ERR_INVALID_ARG),
+    (dict(ws_bytes=100), fa.FA_ERR_INVALID_ARG),
+    (dict(N=-5), fa.FA_ERR_INVALID_ARG),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=-1), fa.FA_ERR_INVALID_ARG),
+])
+def test_bwd_rejects_bad_arguments_without_launching(kw, want):
+    assert _bwd(**kw) == want
+
+
+def test_product_path_does_not_import_oracle():
+    import os
+    import re
+
+    pkg = os.path.dirname(fa.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
