@@ -1,22 +1,478 @@
-// fa_bwd.cuh - attention backward for sm_100a (placeholder until the kernels land).
+// fa_bwd.cuh - attention backward for sm_100a: dO.O row-dot, the main
+// recompute kernel (TMA + tcgen05 + TMEM), and the dQ fp32 -> bf16 convert.
+//
+// Method: "FlashAttention原理：从原始Attention到FlashAttention"
+// (blog.csdn.net/qq_43527718), section 二 "做法" and section 二.5: the forward
+// stores only the softmax normalisation (lse) and the backward recomputes the
+// attention matrix tile by tile on chip instead of reading it from HBM. The
+// gradient formulas are the calculus of the forward:
+//   P = exp(scale*Q K^T - lse),  dV = P^T dO,  dP = dO V^T,
+//   D_i = rowsum(dO_i * O_i),    dS = P * (dP - D),
+//   dQ = scale * dS K,           dK = scale * dS^T Q.
+//
+// Main kernel: one CTA per (batch*head, 128-key tile j); it loops over
+// 64-query tiles i (causal: only i with a visible query, the masked upper
+// triangle is skipped) and keeps dK_j, dV_j accumulating in TMEM. Everything is
+// computed transposed (keys on TMEM lanes) so P^T and dS^T can feed the dV/dK
+// MMAs straight from TMEM:
+//   S^T  = K_j Q_i^T        (SS, M=128 keys, N=64 queries)   -> TMEM S[b]
+//   dP^T = V_j dO_i^T       (SS)                             -> TMEM dP[b]
+//   P^T  = 2^(lambda*S^T - lse2),  dS^T = scale * P^T * (dP^T - D)   (registers)
+//   dV  += P^T dO_i         (TS: A = P^T bf16 in TMEM)
+//   dK  += dS^T Q_i         (TS: A = dS^T bf16 in TMEM)
+//   dQ_i^T = K_j^T dS^T     (SS: A = K_j read MN-major, B = dS from smem)
+//   dQ_i^T is drained from TMEM to shared memory and added into the fp32 dQ
+//   accumulator in global memory with one TMA reduce-add per tile.
+// S and dP are double-buffered (b = iteration & 1) so the tensor core computes
+// tile i+1 while the elementwise warpgroup works on tile i.
+//
+// Roles (320 threads): warp 0 TMA producer (+ lse/D staging), warp 1 MMA
+// issuer, warps 2-5 elementwise warpgroup (thread = key row), warps 6-9 dQ
+// drain warpgroup (thread = head-dim row of dQ^T).
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include "fa.h"
 #include "fa_ptx.cuh"
 
 namespace fa {
 
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   const size_t rows = static_cast<size_t>(BH) * N;
-  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  return up(rows * d * sizeof(float)) + up(rows * sizeof(float));
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-template <typename MakeTile, typename MakeMap>
-fa_status bwd_launch(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
-                     void*, void*, int, int, int, float, int, cudaStream_t, MakeTile, MakeMap) {
-  return FA_ERR_UNSUPPORTED;
+// ------------------------------------------------------------ D = rowsum(dO*O)
+// Also zeroes the fp32 dQ accumulator rows it visits (same rows, same pass).
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dO,
+                                                         float* __restrict__ dsum, float* __restrict__ dq_acc,
+                                                         long long rows) {
+  constexpr int TPR = D / 8;  // threads per row, 16 bytes of each tensor per thread
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int part = static_cast<int>(tid % TPR);
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x / TPR;
+  for (long long row = tid / TPR; row < rows; row += stride) {
+    const size_t off = static_cast<size_t>(row) * D + part * 8;
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
+    const uint4 g = __ldg(reinterpret_cast<const uint4*>(dO + off));
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 af = __bfloat1622float2(a2[e]);
+      const float2 gf = __bfloat1622float2(g2[e]);
+      s = fmaf(af.x, gf.x, s);
+      s = fmaf(af.y, gf.y, s);
+    }
+#pragma unroll
+    for (int w = TPR / 2; w >= 1; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
+    if (part == 0) dsum[row] = s;
+    float4* z = reinterpret_cast<float4*>(dq_acc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// --------------------------------------------------------- dQ fp32 -> bf16
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                __nv_bfloat16* __restrict__ dq, long long n8) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i + 1);
+    uint4 w;
+    w.x = pack_bf16(a.x, a.y);
+    w.y = pack_bf16(a.z, a.w);
+    w.z = pack_bf16(b.x, b.y);
+    w.w = pack_bf16(b.z, b.w);
+    reinterpret_cast<uint4*>(dq)[i] = w;
+  }
+}
+
+// ------------------------------------------------------------------ main kernel
+struct BwdParams {
+  const float* lse;   // [BH, N], natural log
+  const float* dsum;  // [BH, N], rowsum(dO * O)
+  void* dk;           // bf16 [BH, N, D]
+  void* dv;           // bf16 [BH, N, D]
+  int BH;
+  int N;
+  int n_kv;          // ceil(N / 128)
+  int n_q;           // ceil(N / 64)
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kKV = 128 * D * 2;  // K or V tile: 128 keys
+  static constexpr int kQT = 64 * D * 2;   // Q or dO tile: 64 queries
+  static constexpr int kStages = 2;        // Q/dO ring depth
+  static constexpr int kDSTile = 128 * 64 * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kKV;
+  static constexpr int kQ = 2 * kKV;
+  static constexpr int kDO = kQ + kStages * kQT;
+  static constexpr int kDS = kDO + kStages * kQT;  // [2] dS tiles [128 keys][64 queries]
+  static constexpr int kDQ = kDS + 2 * kDSTile;    // fp32 staging [64 queries][D]
+  static constexpr int kStat = kDQ + 64 * D * 4;   // [kStages] x {lse2[64], dsum[64]}
+  static constexpr int kBar = kStat + kStages * 512;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+constexpr int kBwdThreads = 320;
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int QS = L::kStages;
+  constexpr int KCH = D / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* kv_full = bars;
+  uint64_t* qd_full = kv_full + 1;      // [QS]
+  uint64_t* qd_empty = qd_full + QS;    // [QS]
+  uint64_t* s_full = qd_empty + QS;     // [2]
+  uint64_t* dp_full = s_full + 2;       // [2]
+  uint64_t* p_full = dp_full + 2;       // [2]
+  uint64_t* ds_full = p_full + 2;       // [2]
+  uint64_t* dq_full = ds_full + 2;      // [2]
+  uint64_t* dq_empty = dq_full + 2;     // [2]
+  uint64_t* acc_full = dq_empty + 2;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+
+  // Causal: key tile 0 sees every query tile, so low j first (heaviest).
+  int j, bh;
+  if (CAUSAL) {
+    j = static_cast<int>(blockIdx.x) / p.BH;
+    bh = static_cast<int>(blockIdx.x) % p.BH;
+  } else {
+    bh = static_cast<int>(blockIdx.x) / p.n_kv;
+    j = static_cast<int>(blockIdx.x) % p.n_kv;
+  }
+  const int i_start = CAUSAL ? 2 * j : 0;  // first 64-query tile with a visible query
+  const int n_it = p.n_q - i_start;        // >= 1 since 128*j < N
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(qd_full + s, 1);
+      mbar_init(qd_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(dp_full + b, 1);
+      mbar_init(p_full + b, 128);
+      mbar_init(ds_full + b, 128);
+      mbar_init(dq_full + b, 1);
+      mbar_init(dq_empty + b, 128);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S[b] at 64*b, dP[b] at 128 + 64*b, dV at 256, dK at 256 + D.
+  const uint32_t t_dv = 256, t_dk = 256 + D;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    float* stat = reinterpret_cast<float*>(smem + L::kStat);
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_dq);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+      for (int c = 0; c < KCH; ++c) {
+        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, j * 128, bh);
+        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, j * 128, bh);
+      }
+    }
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % QS, u = it / QS;
+      if (it >= QS && !__all_sync(0xffffffffu, wait_parity(qd_empty + s, (u - 1) & 1, abort_flag))) break;
+      const int q0 = (i_start + it) * 64;
+      float* st_lse = stat + s * 128;
+      float* st_d = st_lse + 64;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int qi = q0 + lane + 32 * h;
+        float l2 = 0.f, dd = 0.f;
+        if (qi < N) {
+          const size_t r = static_cast<size_t>(bh) * N + qi;
+          l2 = p.lse[r] * 1.4426950408889634f;
+          dd = p.dsum[r];
+        }
+        st_lse[lane + 32 * h] = l2;
+        st_d[lane + 32 * h] = dd;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(qd_full + s, 2 * L::kQT);
+        for (int c = 0; c < KCH; ++c) {
+          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, q0, bh);
+          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, q0, bh);
+        }
+      }
+      issued = it + 1;
+    }
+    if (lane == 0) {
+      wait_parity_drain(kv_full, 0);
+      for (int it = max(0, issued - QS); it < issued; ++it) wait_parity_drain(qd_full + it % QS, (it / QS) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdST = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T: K-major A and B
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, 0, 1);  // dV, dK: A TMEM, B MN-major
+      constexpr uint32_t kIdDQ = idesc_bf16(D, 64, 1, 1);    // dQ^T: A, B MN-major
+      const uint32_t k_addr = smem_u32(smem + L::kK);
+      const uint32_t v_addr = smem_u32(smem + L::kV);
+      const uint32_t q_addr = smem_u32(smem + L::kQ);
+      const uint32_t do_addr = smem_u32(smem + L::kDO);
+      const uint32_t ds_addr = smem_u32(smem + L::kDS);
+
+      // X^T = A_j Y^T, A_j a 128-row K/V tile, Y a 64-row Q/dO tile (both K-major).
+      auto issue_t = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t ob = (kk >> 2) * 8192 + (kk & 3) * 32;
+          mma_ss(tmem + d_col, sdesc_sw128(a_base + oa, 16, 1024), sdesc_sw128(b_base + ob, 16, 1024), kIdST,
+                 kk > 0);
+        }
+      };
+      // acc += X^T(TMEM, 64 query columns as bf16) * Y (Y a 64-row tile, MN-major)
+      auto issue_acc = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + d_col, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, 8192, 1024), kIdAcc,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dq = [&](int b) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + 128 + 64 * b, sdesc_sw128(k_addr + kk * 2048, 16384, 1024),
+                 sdesc_sw128(ds_addr + b * L::kDSTile + kk * 2048, 8192, 1024), kIdDQ, kk > 0);
+      };
+
+      bool ok = wait_parity(kv_full, 0, abort_flag) && wait_parity(qd_full, 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_t(0, k_addr, q_addr);
+        mma_commit(s_full + 0);
+        issue_t(128, v_addr, do_addr);
+        mma_commit(dp_full + 0);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int b = it & 1, s = it % QS;
+        const int nb = b ^ 1, ns = (it + 1) % QS;
+        const bool has_next = it + 1 < n_it;
+        if (has_next) {
+          if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_t(64 * nb, k_addr, q_addr + ns * L::kQT);
+          mma_commit(s_full + nb);
+        }
+        if (!(ok = wait_parity(p_full + b, (it >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_acc(t_dv, 64 * b, do_addr + s * L::kQT, it > 0);
+        if (has_next) {
+          if (it >= 1 && !(ok = wait_parity(dq_empty + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_t(128 + 64 * nb, v_addr, do_addr + ns * L::kQT);
+          mma_commit(dp_full + nb);
+        }
+        if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_acc(t_dk, 64 * b + 32, q_addr + s * L::kQT, it > 0);
+        issue_dq(b);
+        mma_commit(dq_full + b);
+        mma_commit(qd_empty + s);
+      }
+      if (ok) mma_commit(acc_full);
+      mma_commit(mma_done);
+      wait_parity_drain(mma_done, 0);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------- elementwise (thread = key)
+    const int quarter = warp & 3;
+    const int k = quarter * 32 + lane;
+    const int kj = j * 128 + k;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float* stat = reinterpret_cast<const float*>(smem + L::kStat);
+    const float lam = p.scale_log2;
+    const float scale = p.scale;
+    uint8_t* ds_base = smem + L::kDS;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int b = it & 1, s = it % QS;
+      const int q0 = (i_start + it) * 64;
+      ok = __all_sync(0xffffffffu, wait_parity(qd_full + s, (it / QS) & 1, abort_flag) &&
+                                       wait_parity(s_full + b, (it >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(tmem + lane_off + 64 * b, sv);
+      tmem_ld32(tmem + lane_off + 64 * b + 32, sv + 32);
+      tmem_wait_ld();
+      const float* lse2 = stat + s * 128;
+      const float* dd = lse2 + 64;
+      const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (CAUSAL && j * 128 + 127 > q0);
+      float pr[64];
+#pragma unroll
+      for (int q = 0; q < 64; ++q) pr[q] = ex2(fmaf(__uint_as_float(sv[q]), lam, -lse2[q]));
+      if (edge) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const int qi = q0 + q;
+          const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
+          if (!vis) pr[q] = 0.f;
+        }
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      tmem_st32(tmem + lane_off + 64 * b, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + b);
+
+      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      tmem_ld32(tmem + lane_off + 128 + 64 * b, sv);
+      tmem_ld32(tmem + lane_off + 128 + 64 * b + 32, sv + 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 64; ++q) pr[q] = pr[q] * (__uint_as_float(sv[q]) - dd[q]) * scale;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      tmem_st32(tmem + lane_off + 64 * b + 32, pk);
+      // dS tile b was last read by the dQ MMA two iterations ago.
+      if (it >= 2) {
+        ok = __all_sync(0xffffffffu, wait_parity(dq_full + b, ((it - 2) >> 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      // Row k of the [128 keys][64 queries] tile, 128-byte swizzle.
+      uint8_t* row = ds_base + b * L::kDSTile + k * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(row + ((c ^ (k & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full + b);
+    }
+    // ----------------------------------------------------- dK, dV epilogue
+    if (ok) {
+      ok = __all_sync(0xffffffffu, wait_parity(acc_full, 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const bool valid = kj < N;
+        const size_t row = static_cast<size_t>(bh) * N + (valid ? kj : 0);
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(which ? p.dk : p.dv) + row * D;
+          const uint32_t col = which ? t_dk : t_dv;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + col + c, v);
+            tmem_wait_ld();
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                                    pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                                    pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                                    pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- dQ drain
+    const int quarter = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    // dQ^T rows (head-dim index) held by this thread: M = D = 128 uses every
+    // lane; M = 64 uses lanes 0-15 of each 32-lane quarter.
+    const int drow = (D == 128) ? quarter * 32 + lane : quarter * 16 + lane;
+    const bool holds = (D == 128) || (lane < 16);
+    float* stg = reinterpret_cast<float*>(smem + L::kDQ);
+    const bool leader = (warp == 6 && lane == 0);
+    bool ok = true;
+    // Every drain warp runs all 2*n_it named barriers, even after an abort
+    // (work is skipped instead), so no warp can be left waiting at one.
+    for (int it = 0; it < n_it; ++it) {
+      const int b = it & 1;
+      if (ok) ok = __all_sync(0xffffffffu, wait_parity(dq_full + b, (it >> 1) & 1, abort_flag));
+      uint32_t v[64];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + 128 + 64 * b, v);
+        tmem_ld32(tmem + lane_off + 128 + 64 * b + 32, v + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(dq_empty + b);
+      }
+      if (leader) bulk_wait_group_read0();  // previous reduce has read the staging tile
+      named_bar_sync(1, 128);
+      if (ok && holds) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) stg[q * D + drow] = __uint_as_float(v[q]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (leader && ok) {
+        tma_reduce_add_3d(&tm_dq, stg, 0, (i_start + it) * 64, bh);
+        bulk_commit_group();
+      }
+    }
+    if (leader) bulk_wait_group0();
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 }  // namespace fa

@@ -79,9 +79,21 @@ fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, int d, int N, int
   return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <typename Kern>
-fa_status launch_status(Kern) {
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+fa_status launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+// Grid for the memory-bound helper kernels: enough CTAs to fill every SM a
+// few times over, grid-striding beyond that.
+unsigned helper_grid(long long threads_needed) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const long long blocks = (threads_needed + 255) / 256;
+  const long long cap = static_cast<long long>(sms) * 8;
+  return static_cast<unsigned>(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
 }
 
 template <int D, bool CAUSAL, bool OF32>
@@ -93,7 +105,67 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
   kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, p);
-  return launch_status(kern);
+  return launch_status();
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const fa::BwdParams& p, cudaStream_t st) {
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  const int smem = fa::BwdLayout<D>::kAlloc;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
+  kern<<<grid, fa::kBwdThreads, smem, st>>>(tq, tk, tv, tdo, tdq, p);
+  return launch_status();
+}
+
+template <int D>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* workspace, int BH, int N, float scale, int causal,
+                     cudaStream_t st) {
+  const long long rows = static_cast<long long>(BH) * N;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + fa::align256(rows * D * sizeof(float)));
+
+  // 1. D = rowsum(dO * O) and dQ accumulator = 0.
+  fa::fa_bwd_dot_kernel<D><<<helper_grid(rows * (D / 8)), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), dsum, dq_acc, rows);
+  fa_status s = launch_status();
+  if (s != FA_OK) return s;
+
+  // 2. Main kernel.
+  alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
+  if ((s = make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+      FA_OK)
+    return s;
+  if ((s = make_tmap(&tdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+    return s;
+  if ((s = make_bf16_tile_map(&tk, k, D, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tv, v, D, N, BH)) != FA_OK) return s;
+  if ((s = make_tmap(&tdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+      FA_OK)
+    return s;
+  fa::BwdParams p;
+  p.lse = lse;
+  p.dsum = dsum;
+  p.dk = dk;
+  p.dv = dv;
+  p.BH = BH;
+  p.N = N;
+  p.n_kv = (N + 127) / 128;
+  p.n_q = (N + 63) / 64;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  s = causal ? launch_bwd_main<D, true>(tq, tk, tv, tdo, tdq, p, st)
+             : launch_bwd_main<D, false>(tq, tk, tv, tdo, tdq, p, st);
+  if (s != FA_OK) return s;
+
+  // 3. dq = bf16(dQ accumulator).
+  const long long n8 = rows * D / 8;
+  fa::fa_bwd_dq_convert_kernel<<<helper_grid(n8), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  return launch_status();
 }
 
 }  // namespace
@@ -161,8 +233,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (s != FA_OK) return s;
   if (ws_bytes < fa::bwd_workspace_bytes(B * H, N, d)) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
-  return fa::bwd_launch(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, d, scale, causal,
-                        static_cast<cudaStream_t>(stream), make_bf16_tile_map, make_tmap);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
 }
 
 fa_status fa_get_device_error(void* stream) {
