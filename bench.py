@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused attention library on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input
+of the headline workload, B=1, H=16, N=16384, d=128 (bf16 inputs): forward and
+backward without a mask, then forward and backward with the causal mask.
+That is four C-ABI calls and eight kernel launches. The metric is
+attention TFLOPS/s, counted as 4*B*H*N^2*d for the forward and 2.5x that for
+the backward, each halved under the causal mask.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0). With N > 1 (launched by torch.distributed.run)
+every rank runs an independent replica of the workload: the path needs no
+exchange between GPUs, so there is no data-path collective; the only
+collectives are the barrier and the max-over-ranks of the timed region.
+
+--impl reference times the fp64 CPU oracle (the slow, plainly correct
+definition of the same computation) on the host cores, on a bounded sample of
+the same workload each step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPS/s on 1 B200 at N=16k d=128; % of bf16 tensor peak"
+UNIT = "TFLOPS/s"
+B, H, N, D = 1, 16, 16384, 128
+SEED = 3
+WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then causal"
+
+# DRAM traffic of the main backward kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum per launch, non-causal launch
+# of the workload above). Valid only for the kernel source it was taken on.
+BWD_TRAFFIC = {"bytes": None, "source_sha256": None, "profile": None}
+
+
+def _flops(causal: bool):
+    f = 4.0 * B * H * N * N * D
+    f = f / 2 if causal else f
+    return f, 2.5 * f
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            m = json.load(fh)
+        return float(m["bf16_tflops"]), float(m.get("bf16_tflops_sustained", m["bf16_tflops"])), \
+            float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _bwd_source_sha():
+    h = hashlib.sha256()
+    for f in ("fa_bwd.cuh", "fa_ptx.cuh"):
+        with open(os.path.join(ROOT, "exact_attention_118_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of one GPU during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", gpu_index], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ oracle sample
+
+def _visible_pairs(rows, causal):
+    rows = list(rows)
+    return sum(r + 1 for r in rows) if causal else len(rows) * N
+
+
+def oracle_sample(x, head, rows):
+    """Time the fp64 oracle on query rows `rows` of one head, forward and
+    backward, non-causal and causal. Returns (seconds, algorithmic FLOPs)."""
+    from oracle import attention_backward_rows, attention_forward_rows
+
+    flops = 0.0
+    t0 = time.perf_counter()
+    for causal in (False, True):
+        attention_forward_rows(x["q"], x["k"], x["v"], D ** -0.5, causal, [head], rows)
+        attention_backward_rows(x["q"], x["k"], x["v"], x["do"], D ** -0.5, causal, [head], rows)
+        flops += 4.0 * D * _visible_pairs(rows, causal) * 3.5  # forward + 2.5x backward
+    return time.perf_counter() - t0, flops
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args):
+    """fp64 CPU oracle, one bounded sample of the workload per step."""
+    from workloads import make_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = make_inputs(B, H, N, D, SEED)  # the workload's own inputs; the sample uses head (0, 0)
+    rows_per_step = 512
+    for _ in range(args.warmup):
+        oracle_sample(x, (0, 0), range(0, rows_per_step))
+    total_t, total_f = 0.0, 0.0
+    for s in range(args.steps):
+        r0 = (s * rows_per_step) % N
+        dt, f = oracle_sample(x, (0, 0), range(r0, r0 + rows_per_step))
+        total_t += dt
+        total_f += f
+    value = total_f / total_t / 1e12
+    cores = _cpu_threads()
+    sample = (f"query rows of head (0,0), {rows_per_step} rows per step "
+              f"(rows {0}..{(args.steps * rows_per_step) % N or N}), forward+backward, non-causal and causal")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": N, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_118_b200 as fa
+    from workloads import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # CPU baseline first (rank 0, one GPU only), before the GPU is busy.
+    cpu_baseline = None
+    x_cpu = make_inputs(B, H, N, D, SEED)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = range(0, 4096)
+        dt, f = oracle_sample(x_cpu, (0, 0), rows)
+        cpu_baseline = {"value": f / dt / 1e12, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+                        "sample": "query rows 0..4095 of head (0,0), forward+backward, non-causal and causal "
+                                  f"({dt:.1f} s)"}
+
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    # Pinned host copies of the step's inputs (for the end-to-end number) and
+    # their device-resident counterparts.
+    host_in = {k: v.pin_memory() for k, v in x_cpu.items()}
+    dev_in = {k: v.to(dev) for k, v in host_in.items()}
+    shape = (B, H, N, D)
+
+    def outputs():
+        return {
+            "o": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+            "lse": torch.empty((B, H, N), dtype=torch.float32, device=dev),
+            "dq": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+            "dk": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+            "dv": torch.empty(shape, dtype=torch.bfloat16, device=dev),
+        }
+
+    outs = {False: outputs(), True: outputs()}
+    ws_bytes = fa.fa_bwd_workspace_size(B, H, N, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scale = D ** -0.5
+    q, k, v, do = (dev_in[n].data_ptr() for n in ("q", "k", "v", "do"))
+
+    def check(st, what):
+        if st != fa.FA_OK:
+            raise RuntimeError(f"{what}: {fa.fa_strerror(st)}")
+
+    def run_pass(causal, ev=None):
+        o = outs[causal]
+        check(fa.fa_fwd(q, k, v, o["o"].data_ptr(), o["lse"].data_ptr(), B, H, N, D, scale, int(causal),
+                        fa.FA_BF16, sp), "fa_fwd")
+        if ev is not None:
+            ev[0].record(stream)
+            fa.fa_set_bwd_main_events(ev[1].cuda_event, ev[2].cuda_event)
+        check(fa.fa_bwd(q, k, v, o["o"].data_ptr(), o["lse"].data_ptr(), do, o["dq"].data_ptr(),
+                        o["dk"].data_ptr(), o["dv"].data_ptr(), ws.data_ptr(), ws_bytes, B, H, N, D, scale,
+                        int(causal), sp), "fa_bwd")
+        if ev is not None:
+            fa.fa_set_bwd_main_events(None, None)
+            ev[3].record(stream)
+
+    def step(evs=None):
+        run_pass(False, None if evs is None else evs[0])
+        run_pass(True, None if evs is None else evs[1])
+
+    fwd_nc, bwd_nc = _flops(False)
+    fwd_c, bwd_c = _flops(True)
+    step_flops = fwd_nc + bwd_nc + fwd_c + bwd_c
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    check(fa.fa_get_device_error(sp), "warm-up")
+
+    # ---------------------------------------------- device-resident timed region
+    def mk():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)  # creates the underlying cudaEvent_t
+        return e
+
+    evs = [[[mk() for _ in range(4)] for _ in range(2)] for _ in range(args.steps)]
+    gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local] if os.environ.get(
+        "CUDA_VISIBLE_DEVICES") else str(local)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    start, stop = mk(), mk()
+    start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    check(fa.fa_get_device_error(sp), "timed region")
+    ms_total = max_over_ranks(start.elapsed_time(stop))
+    ms_per_step = ms_total / args.steps
+    value = step_flops * world / (ms_per_step / 1e3) / 1e12
+
+    # per-pass breakdown (events around each call) and the main backward kernel
+    def med(xs):
+        return statistics.median(xs)
+
+    per = {}
+    bwd_main_ms = {False: [], True: []}
+    for c in (False, True):
+        e = [evs[s][int(c)] for s in range(args.steps)]
+        bwd_total = [x[0].elapsed_time(x[3]) for x in e]
+        main = [x[1].elapsed_time(x[2]) for x in e]
+        bwd_main_ms[c] = main
+        per[c] = {"bwd_ms": med(bwd_total), "bwd_main_ms": med(main)}
+
+    # forward alone, timed the same way in its own loop
+    fwd_ms = {}
+    for c in (False, True):
+        o = outs[c]
+        a, b_ = mk(), mk()
+        a.record(stream)
+        for _ in range(args.steps):
+            check(fa.fa_fwd(q, k, v, o["o"].data_ptr(), o["lse"].data_ptr(), B, H, N, D, scale, int(c),
+                            fa.FA_BF16, sp), "fa_fwd")
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        fwd_ms[c] = a.elapsed_time(b_) / args.steps
+
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    passes = {}
+    for c, tag in ((False, "noncausal"), (True, "causal")):
+        ff, fb = _flops(c)
+        passes[f"fwd_{tag}"] = {"ms": fwd_ms[c], "tflops": ff / fwd_ms[c] / 1e9,
+                                "frac_of_peak": ff / fwd_ms[c] / 1e9 / peak}
+        passes[f"bwd_{tag}"] = {"ms": per[c]["bwd_ms"], "tflops": fb / per[c]["bwd_ms"] / 1e9,
+                                "frac_of_peak": fb / per[c]["bwd_ms"] / 1e9 / peak,
+                                "main_kernel_ms": per[c]["bwd_main_ms"]}
+
+    # Roofline of the dominant kernel: the main backward kernel (both masks).
+    main_total_ms = sum(bwd_main_ms[False]) + sum(bwd_main_ms[True])
+    main_flops = args.steps * (bwd_nc + bwd_c)
+    achieved = main_flops / (main_total_ms / 1e3) / 1e12
+    traffic = None
+    if BWD_TRAFFIC["bytes"] is not None and BWD_TRAFFIC["source_sha256"] == _bwd_source_sha():
+        traffic = BWD_TRAFFIC["bytes"]
+    roofline = {"kernel": "fa_bwd_kernel<128> (main backward)", "bound": "tensor", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_kind": f"{peak_kind} bf16 dense (burst); sustained {peak_sus}",
+                "frac_of_sustained": achieved / peak_sus}
+
+    # ---------------------------------------------------- end-to-end (host buffers)
+    host_out = {c: {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs[c].items()}
+                for c in (False, True)}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for c in (False, True) for t in host_out[c].values())
+
+    def e2e_step():
+        for n in ("q", "k", "v", "do"):
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        step()
+        for c in (False, True):
+            for n, t in outs[c].items():
+                host_out[c][n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    a, b_ = mk(), mk()
+    a.record(stream)
+    e2e_steps = max(1, min(args.steps, 10))
+    for _ in range(e2e_steps):
+        e2e_step()
+    b_.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(a.elapsed_time(b_)) / e2e_steps
+    check(fa.fa_get_device_error(sp), "e2e")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": N, "heads": H, "head_dim": D,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (Q,K,V,dO 67 MB each; 1.1 GB working set per step)"},
+        "frac_of_peak": value / peak,
+        "passes": passes,
+        "roofline": roofline,
+        "cpu_baseline": cpu_baseline,
+        "e2e": {"value": step_flops * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clocks,
+        "context": "pages' figure: FlashAttention-2 ~338 TFLOPS/s non-causal at 16k on H100 SXM5 (other hardware)",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,7 +1,8 @@
 """Python binding of libfa.so: exact, IO-aware fused attention for B200 (sm_100a).
 
 The functions ``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_size``,
-``fa_get_device_error``, ``fa_strerror`` and ``fa_version`` have the names and
+``fa_get_device_error``, ``fa_set_bwd_main_events``, ``fa_last_cuda_error``,
+``fa_strerror`` and ``fa_version`` have the names and
 arguments of the C ABI in ``include/fa.h`` (pointers and the stream are plain
 integers) and only marshal arguments. ``attention_forward`` and
 ``attention_backward`` are conveniences that take torch CUDA tensors, allocate
@@ -33,6 +34,8 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "fa_get_device_error": (_I, [_P]),
+    "fa_set_bwd_main_events": (_I, [_P, _P]),
+    "fa_last_cuda_error": (_I, []),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -41,7 +44,7 @@ _SIGNATURES = {
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m exact_attention_118_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python exact_attention_118_b200/build.py` "
             "(nvcc, sm_100a). There is no fallback path."
         )
     lib = ctypes.CDLL(LIB_PATH)
@@ -64,7 +67,8 @@ def header_symbols():
 
 class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {fa_strerror(status)} (status {status})")
+        extra = f", cuda error {fa_last_cuda_error()}" if status == FA_ERR_CUDA else ""
+        super().__init__(f"{what}: {fa_strerror(status)} (status {status}{extra})")
         self.status = status
 
 
@@ -84,6 +88,14 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, sca
 
 def fa_get_device_error(stream) -> int:
     return _lib.fa_get_device_error(stream)
+
+
+def fa_set_bwd_main_events(before, after) -> int:
+    return _lib.fa_set_bwd_main_events(before, after)
+
+
+def fa_last_cuda_error() -> int:
+    return _lib.fa_last_cuda_error()
 
 
 def fa_strerror(status: int) -> str:

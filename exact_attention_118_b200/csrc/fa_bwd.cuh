@@ -24,11 +24,13 @@
 //   dQ_i^T is drained from TMEM to shared memory and added into the fp32 dQ
 //   accumulator in global memory with one TMA reduce-add per tile.
 // S and dP are double-buffered (b = iteration & 1) so the tensor core computes
-// tile i+1 while the elementwise warpgroup works on tile i.
+// tile i+1 while an elementwise warpgroup works on tile i; each buffer has its
+// own elementwise warpgroup, so the two groups overlap each other's waits.
 //
-// Roles (320 threads): warp 0 TMA producer (+ lse/D staging), warp 1 MMA
-// issuer, warps 2-5 elementwise warpgroup (thread = key row), warps 6-9 dQ
-// drain warpgroup (thread = head-dim row of dQ^T).
+// Roles (512 threads): warp 0 TMA producer (Q, dO, lse2 and D tiles), warp 1
+// MMA issuer, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
+// dQ^T), warps 8-11 and 12-15 two elementwise warpgroups (thread = key row)
+// that take alternate query tiles.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -38,18 +40,29 @@ namespace fa {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Row stride (elements) of the per-row statistics in the workspace: N rounded
+// up to a multiple of 4 so each row starts on a 16-byte boundary (TMA rule).
+inline int stat_stride(int N) { return (N + 3) & ~3; }
+
+// Workspace: [dQ accumulator fp32 BH*N*d][lse2 fp32 BH*Np][D fp32 BH*Np],
+// each piece starting on a 256-byte boundary (Np = stat_stride(N)).
 inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   const size_t rows = static_cast<size_t>(BH) * N;
-  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+  const size_t srows = static_cast<size_t>(BH) * stat_stride(N);
+  return align256(rows * d * sizeof(float)) + 2 * align256(srows * sizeof(float));
 }
 
-// ------------------------------------------------------------ D = rowsum(dO*O)
-// Also zeroes the fp32 dQ accumulator rows it visits (same rows, same pass).
+// ------------------------------------------------- D = rowsum(dO*O), lse2
+// For every query row: D = sum_k dO_k * O_k, lse2 = lse * log2(e) (the
+// forward's natural-log normaliser moved to base 2 for the exp2 recompute),
+// both written with the padded row stride Np; and the row of the fp32 dQ
+// accumulator is zeroed (same rows, same pass).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
+                                                         const float* __restrict__ lse, float* __restrict__ lse2,
                                                          float* __restrict__ dsum, float* __restrict__ dq_acc,
-                                                         long long rows) {
+                                                         long long rows, int N, int Np) {
   constexpr int TPR = D / 8;  // threads per row, 16 bytes of each tensor per thread
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int part = static_cast<int>(tid % TPR);
@@ -70,7 +83,12 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __
     }
 #pragma unroll
     for (int w = TPR / 2; w >= 1; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
-    if (part == 0) dsum[row] = s;
+    if (part == 0) {
+      const long long bh = row / N, qi = row - bh * N;
+      const size_t so = static_cast<size_t>(bh) * Np + qi;
+      dsum[so] = s;
+      lse2[so] = __ldg(lse + row) * 1.4426950408889634f;
+    }
     float4* z = reinterpret_cast<float4*>(dq_acc + off);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -95,10 +113,8 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
 
 // ------------------------------------------------------------------ main kernel
 struct BwdParams {
-  const float* lse;   // [BH, N], natural log
-  const float* dsum;  // [BH, N], rowsum(dO * O)
-  void* dk;           // bf16 [BH, N, D]
-  void* dv;           // bf16 [BH, N, D]
+  void* dk;  // bf16 [BH, N, D]
+  void* dv;  // bf16 [BH, N, D]
   int BH;
   int N;
   int n_kv;          // ceil(N / 128)
@@ -109,9 +125,9 @@ struct BwdParams {
 
 template <int D>
 struct BwdLayout {
-  static constexpr int kKV = 128 * D * 2;  // K or V tile: 128 keys
-  static constexpr int kQT = 64 * D * 2;   // Q or dO tile: 64 queries
-  static constexpr int kStages = 2;        // Q/dO ring depth
+  static constexpr int kKV = 128 * D * 2;          // K or V tile: 128 keys
+  static constexpr int kQT = 64 * D * 2;           // Q or dO tile: 64 queries
+  static constexpr int kStages = (D == 128) ? 3 : 4;  // Q/dO/lse2/D ring depth
   static constexpr int kDSTile = 128 * 64 * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kKV;
@@ -119,14 +135,22 @@ struct BwdLayout {
   static constexpr int kDO = kQ + kStages * kQT;
   static constexpr int kDS = kDO + kStages * kQT;  // [2] dS tiles [128 keys][64 queries]
   static constexpr int kDQ = kDS + 2 * kDSTile;    // fp32 staging [64 queries][D]
-  static constexpr int kStat = kDQ + 64 * D * 4;   // [kStages] x {lse2[64], dsum[64]}
+  static constexpr int kStat = kDQ + 64 * D * 4;   // [kStages] x {lse2[64], D[64]}
   static constexpr int kBar = kStat + kStages * 512;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-constexpr int kBwdThreads = 320;
+// Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warp 1
+// MMA issuer and TMEM owner, warps 2-3 idle), 4-7 dQ drain, 8-11 elementwise
+// (even iterations, TMEM buffer 0), 12-15 elementwise (odd iterations, buffer
+// 1). Launched at 128 registers per thread (512 x 128 = the 64K register
+// file; each SM sub-partition holds one warp of every warpgroup); the groups
+// then move to 56 / 104 / 176 / 176, which sums to the same 512 per slot.
+constexpr int kBwdThreads = 512;
+constexpr int kRegCtl = 56, kRegDrain = 104, kRegElem = 176;
+static_assert(kRegCtl + kRegDrain + 2 * kRegElem == 512, "register split must equal the launch budget");
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -136,7 +160,8 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_lse2,
+                  const __grid_constant__ CUtensorMap tm_dsum, const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kStages;
   constexpr int KCH = D / 64;
@@ -184,10 +209,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       mbar_init(dp_full + b, 1);
-      mbar_init(p_full + b, 128);
-      mbar_init(ds_full + b, 128);
+      mbar_init(p_full + b, 4);   // one arrival per warp of the elementwise group
+      mbar_init(ds_full + b, 4);
       mbar_init(dq_full + b, 1);
-      mbar_init(dq_empty + b, 128);
+      mbar_init(dq_empty + b, 4);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
@@ -199,54 +224,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int wg = warp >> 2;
   // TMEM columns: S[b] at 64*b, dP[b] at 128 + 64*b, dV at 256, dK at 256 + D.
   const uint32_t t_dv = 256, t_dk = 256 + D;
+  constexpr uint32_t kStageTx = 2 * L::kQT + 512;
 
+  if (wg == 0) setmaxnreg_dec<kRegCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    float* stat = reinterpret_cast<float*>(smem + L::kStat);
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_dq);
+      prefetch_tmap(&tm_lse2);
+      prefetch_tmap(&tm_dsum);
       mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
       for (int c = 0; c < KCH; ++c) {
         tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, j * 128, bh);
         tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, j * 128, bh);
       }
-    }
-    int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it % QS, u = it / QS;
-      if (it >= QS && !__all_sync(0xffffffffu, wait_parity(qd_empty + s, (u - 1) & 1, abort_flag))) break;
-      const int q0 = (i_start + it) * 64;
-      float* st_lse = stat + s * 128;
-      float* st_d = st_lse + 64;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int qi = q0 + lane + 32 * h;
-        float l2 = 0.f, dd = 0.f;
-        if (qi < N) {
-          const size_t r = static_cast<size_t>(bh) * N + qi;
-          l2 = p.lse[r] * 1.4426950408889634f;
-          dd = p.dsum[r];
-        }
-        st_lse[lane + 32 * h] = l2;
-        st_d[lane + 32 * h] = dd;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(qd_full + s, 2 * L::kQT);
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it % QS, u = it / QS;
+        if (it >= QS && !wait_parity(qd_empty + s, (u - 1) & 1, abort_flag)) break;
+        const int q0 = (i_start + it) * 64;
+        uint8_t* st = smem + L::kStat + s * 512;
+        mbar_arrive_expect_tx(qd_full + s, kStageTx);
         for (int c = 0; c < KCH; ++c) {
           tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, q0, bh);
           tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, q0, bh);
         }
+        tma_load_2d(st, &tm_lse2, qd_full + s, q0, bh);
+        tma_load_2d(st + 256, &tm_dsum, qd_full + s, q0, bh);
+        issued = it + 1;
       }
-      issued = it + 1;
-    }
-    if (lane == 0) {
       wait_parity_drain(kv_full, 0);
       for (int it = max(0, issued - QS); it < issued; ++it) wait_parity_drain(qd_full + it % QS, (it / QS) & 1);
     }
@@ -324,108 +336,132 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(mma_done);
       wait_parity_drain(mma_done, 0);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------- elementwise (thread = key)
+  } else if (wg >= 2) {
+    // ---------------------------------------- elementwise (thread = key row)
+    // Group e handles iterations it = e, e+2, ... with TMEM/smem buffer b = e.
+    setmaxnreg_inc<kRegElem>();
+    const int e = wg - 2;
     const int quarter = warp & 3;
     const int k = quarter * 32 + lane;
     const int kj = j * 128 + k;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float* stat = reinterpret_cast<const float*>(smem + L::kStat);
     const float lam = p.scale_log2;
     const float scale = p.scale;
-    uint8_t* ds_base = smem + L::kDS;
+    const int b = e;
+    const uint32_t tS = tmem + lane_off + 64 * b;
+    const uint32_t tP = tmem + lane_off + 128 + 64 * b;
+    uint8_t* ds_row = smem + L::kDS + b * L::kDSTile + k * 128;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int b = it & 1, s = it % QS;
+    for (int it = e; it < n_it; it += 2) {
+      const int s = it % QS;
       const int q0 = (i_start + it) * 64;
       ok = __all_sync(0xffffffffu, wait_parity(qd_full + s, (it / QS) & 1, abort_flag) &&
                                        wait_parity(s_full + b, (it >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(tmem + lane_off + 64 * b, sv);
-      tmem_ld32(tmem + lane_off + 64 * b + 32, sv + 32);
-      tmem_wait_ld();
-      const float* lse2 = stat + s * 128;
-      const float* dd = lse2 + 64;
+      const float4* lse2 = reinterpret_cast<const float4*>(smem + L::kStat + s * 512);
+      const float4* dd = lse2 + 16;
       const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (CAUSAL && j * 128 + 127 > q0);
       float pr[64];
 #pragma unroll
-      for (int q = 0; q < 64; ++q) pr[q] = ex2(fmaf(__uint_as_float(sv[q]), lam, -lse2[q]));
-      if (edge) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[32];
+        tmem_ld32(tS + 32 * h, sv);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          const int qi = q0 + q;
-          const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
-          if (!vis) pr[q] = 0.f;
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = lse2[8 * h + c4];
+          const int q = 32 * h + 4 * c4;
+          pr[q + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), lam, -l4.x));
+          pr[q + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), lam, -l4.y));
+          pr[q + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), lam, -l4.z));
+          pr[q + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), lam, -l4.w));
         }
-      }
-      uint32_t pk[32];
+        if (edge) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-      tmem_st32(tmem + lane_off + 64 * b, pk);
+          for (int c = 0; c < 32; ++c) {
+            const int qi = q0 + 32 * h + c;
+            const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
+            if (!vis) pr[32 * h + c] = 0.f;
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(pr[32 * h + 2 * c], pr[32 * h + 2 * c + 1]);
+        tmem_st16(tS + 16 * h, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full + b);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + b);
 
-      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag));
+      // dS tile b was last read by the dQ MMA of iteration it - 2.
+      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag) &&
+                                       (it < 2 || wait_parity(dq_full + b, ((it - 2) >> 1) & 1, abort_flag)));
       if (!ok) break;
       tc_fence_after();
-      tmem_ld32(tmem + lane_off + 128 + 64 * b, sv);
-      tmem_ld32(tmem + lane_off + 128 + 64 * b + 32, sv + 32);
-      tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 64; ++q) pr[q] = pr[q] * (__uint_as_float(sv[q]) - dd[q]) * scale;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t dp[32];
+        tmem_ld32(tP + 32 * h, dp);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-      tmem_st32(tmem + lane_off + 64 * b + 32, pk);
-      // dS tile b was last read by the dQ MMA two iterations ago.
-      if (it >= 2) {
-        ok = __all_sync(0xffffffffu, wait_parity(dq_full + b, ((it - 2) >> 1) & 1, abort_flag));
-        if (!ok) break;
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 d4 = dd[8 * h + c4];
+          const int q = 32 * h + 4 * c4;
+          const float s0 = pr[q + 0] * (__uint_as_float(dp[4 * c4 + 0]) - d4.x) * scale;
+          const float s1 = pr[q + 1] * (__uint_as_float(dp[4 * c4 + 1]) - d4.y) * scale;
+          const float s2 = pr[q + 2] * (__uint_as_float(dp[4 * c4 + 2]) - d4.z) * scale;
+          const float s3 = pr[q + 3] * (__uint_as_float(dp[4 * c4 + 3]) - d4.w) * scale;
+          pk[2 * c4] = pack_bf16(s0, s1);
+          pk[2 * c4 + 1] = pack_bf16(s2, s3);
+        }
+        tmem_st16(tS + 32 + 16 * h, pk);
+        // Row k of the [128 keys][64 queries] dS tile, 128-byte swizzle:
+        // 16-byte chunk c (queries 8c..8c+7) lives at chunk c ^ (k & 7).
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * h + c;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (k & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
       }
-      // Row k of the [128 keys][64 queries] tile, 128-byte swizzle.
-      uint8_t* row = ds_base + b * L::kDSTile + k * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(row + ((c ^ (k & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full + b);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full + b);
     }
-    // ----------------------------------------------------- dK, dV epilogue
+    // -------------------------------------- epilogue: group 0 dV, group 1 dK
     if (ok) {
       ok = __all_sync(0xffffffffu, wait_parity(acc_full, 0, abort_flag));
       if (ok) {
         tc_fence_after();
         const bool valid = kj < N;
         const size_t row = static_cast<size_t>(bh) * N + (valid ? kj : 0);
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e ? p.dk : p.dv) + row * D;
+        const uint32_t col = e ? t_dk : t_dv;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(which ? p.dk : p.dv) + row * D;
-          const uint32_t col = which ? t_dk : t_dv;
+        for (int c = 0; c < D; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + col + c, v);
+          tmem_wait_ld();
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + col + c, v);
-            tmem_wait_ld();
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(out + c);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                                    pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                                    pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                                    pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-            }
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                                  pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                                  pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                                  pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
           }
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------- dQ drain
+  } else if (wg == 1) {
+    // ------------------------------------------------- dQ drain (warps 4-7)
+    setmaxnreg_dec<kRegDrain>();
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     // dQ^T rows (head-dim index) held by this thread: M = D = 128 uses every
@@ -433,7 +469,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int drow = (D == 128) ? quarter * 32 + lane : quarter * 16 + lane;
     const bool holds = (D == 128) || (lane < 16);
     float* stg = reinterpret_cast<float*>(smem + L::kDQ);
-    const bool leader = (warp == 6 && lane == 0);
+    const bool leader = (warp == 4 && lane == 0);
     bool ok = true;
     // Every drain warp runs all 2*n_it named barriers, even after an abort
     // (work is skipped instead), so no warp can be left waiting at one.
@@ -447,7 +483,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tmem + lane_off + 128 + 64 * b + 32, v + 32);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(dq_empty + b);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_empty + b);
       }
       if (leader) bulk_wait_group_read0();  // previous reduce has read the staging tile
       named_bar_sync(1, 128);

@@ -20,6 +20,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn g_encode = nullptr;
+// Reported by fa_last_cuda_error when a TMA descriptor could not be encoded.
+constexpr int kEncodeFailed = -1;
+thread_local int t_last_cuda_error = 0;
 std::once_flag g_encode_once;
 
 EncodeTiledFn encode_fn() {
@@ -72,6 +75,7 @@ fa_status make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) t_last_cuda_error = kEncodeFailed;
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -79,7 +83,22 @@ fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, int d, int N, int
   return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-fa_status launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+// Caller-provided events recorded around the main backward kernel
+// (fa_set_bwd_main_events); per host thread.
+thread_local cudaEvent_t t_bwd_ev_before = nullptr;
+thread_local cudaEvent_t t_bwd_ev_after = nullptr;
+
+fa_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return FA_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+fa_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
 
 // Grid for the memory-bound helper kernels: enough CTAs to fill every SM a
 // few times over, grid-striding beyond that.
@@ -101,23 +120,41 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      cudaStream_t st) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, OF32>;
   const int smem = fa::FwdLayout<D>::kAlloc;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return FA_ERR_CUDA;
+  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+    return cuda_fail(e);
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
   kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, p);
   return launch_status();
 }
 
+// 2-D fp32 map of a [BH][Np] statistics array (Np >= N, a multiple of 4),
+// dims {N, BH}: a 64-wide row box, zero-filled past N.
+fa_status make_stat_map(CUtensorMap* m, const float* base, int N, int Np, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Np) * 4};
+  const cuuint32_t box[2] = {64u, 1u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) t_last_cuda_error = kEncodeFailed;
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D, bool CAUSAL>
-fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tdo, const CUtensorMap& tdq, const fa::BwdParams& p, cudaStream_t st) {
+fa_status launch_bwd_main(const CUtensorMap* maps, const fa::BwdParams& p, cudaStream_t st) {
   auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
   const int smem = fa::BwdLayout<D>::kAlloc;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return FA_ERR_CUDA;
+  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+    return cuda_fail(e);
   const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
-  kern<<<grid, fa::kBwdThreads, smem, st>>>(tq, tk, tv, tdo, tdq, p);
-  return launch_status();
+  if (t_bwd_ev_before && cudaEventRecord(t_bwd_ev_before, st) != cudaSuccess) return FA_ERR_CUDA;
+  kern<<<grid, fa::kBwdThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
+  const fa_status s = launch_status();
+  if (s == FA_OK && t_bwd_ev_after && cudaEventRecord(t_bwd_ev_after, st) != cudaSuccess) return FA_ERR_CUDA;
+  return s;
 }
 
 template <int D>
@@ -125,31 +162,36 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      void* dq, void* dk, void* dv, void* workspace, int BH, int N, float scale, int causal,
                      cudaStream_t st) {
   const long long rows = static_cast<long long>(BH) * N;
-  float* dq_acc = static_cast<float*>(workspace);
-  float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + fa::align256(rows * D * sizeof(float)));
+  const int Np = fa::stat_stride(N);
+  char* ws = static_cast<char*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + fa::align256(rows * D * sizeof(float)));
+  float* dsum = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) +
+                                         fa::align256(static_cast<size_t>(BH) * Np * sizeof(float)));
 
-  // 1. D = rowsum(dO * O) and dQ accumulator = 0.
+  // 1. D = rowsum(dO * O), lse2 = lse * log2(e), dQ accumulator = 0.
   fa::fa_bwd_dot_kernel<D><<<helper_grid(rows * (D / 8)), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), dsum, dq_acc, rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dsum, dq_acc, rows,
+      N, Np);
   fa_status s = launch_status();
   if (s != FA_OK) return s;
 
-  // 2. Main kernel.
-  alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
-  if ((s = make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
-      FA_OK)
-    return s;
-  if ((s = make_tmap(&tdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
+  // 2. Main kernel. Maps: q, k, v, dO, dQ accumulator, lse2, D.
+  alignas(64) CUtensorMap maps[7];
+  if ((s = make_tmap(&maps[0], q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
-  if ((s = make_bf16_tile_map(&tk, k, D, N, BH)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&tv, v, D, N, BH)) != FA_OK) return s;
-  if ((s = make_tmap(&tdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
-      FA_OK)
+  if ((s = make_bf16_tile_map(&maps[1], k, D, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&maps[2], v, D, N, BH)) != FA_OK) return s;
+  if ((s = make_tmap(&maps[3], dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
+  if ((s = make_tmap(&maps[4], dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 64,
+                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+    return s;
+  if ((s = make_stat_map(&maps[5], lse2, N, Np, BH)) != FA_OK) return s;
+  if ((s = make_stat_map(&maps[6], dsum, N, Np, BH)) != FA_OK) return s;
   fa::BwdParams p;
-  p.lse = lse;
-  p.dsum = dsum;
   p.dk = dk;
   p.dv = dv;
   p.BH = BH;
@@ -158,8 +200,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.n_q = (N + 63) / 64;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  s = causal ? launch_bwd_main<D, true>(tq, tk, tv, tdo, tdq, p, st)
-             : launch_bwd_main<D, false>(tq, tk, tv, tdo, tdq, p, st);
+  s = causal ? launch_bwd_main<D, true>(maps, p, st) : launch_bwd_main<D, false>(maps, p, st);
   if (s != FA_OK) return s;
 
   // 3. dq = bf16(dQ accumulator).
@@ -236,6 +277,14 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
   return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+fa_status fa_set_bwd_main_events(void* before, void* after) {
+  t_bwd_ev_before = static_cast<cudaEvent_t>(before);
+  t_bwd_ev_after = static_cast<cudaEvent_t>(after);
+  return FA_OK;
 }
 
 fa_status fa_get_device_error(void* stream) {

@@ -74,8 +74,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * Bytes of caller-owned device workspace fa_bwd needs: a fp32 [B,H,N,d]
- * accumulator for dQ plus the fp32 [B,H,N] row-dot D = rowsum(dO * O),
- * rounded up to 256-byte pieces. Returns 0 for invalid sizes.
+ * accumulator for dQ, then two fp32 [B,H,N'] per-row arrays (lse in base 2,
+ * and the row-dot D = rowsum(dO * O)) with N' = N rounded up to a multiple of
+ * 4; each piece rounded up to 256 bytes. Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -85,10 +86,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *     dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO_i * O_i),
  *     dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q,
  * with P recomputed on chip from q, k and lse (blog section 二.5, second point).
- * Launches, in order on `stream`: a memset of the dQ accumulator, the dO.O
- * row-dot kernel, the main kernel (loops over query tiles for each key tile,
- * accumulating dK and dV on chip and adding dQ contributions into the fp32
- * accumulator), and a kernel that converts the accumulator to bf16 dq.
+ * Launches three kernels, in order on `stream`: the dO.O row-dot kernel
+ * (which also zeroes the dQ accumulator), the main kernel (loops over query
+ * tiles for each key tile, accumulating dK and dV on chip and adding dQ
+ * contributions into the fp32 accumulator), and a kernel that converts the
+ * accumulator to bf16 dq.
  * workspace: device pointer, 256-byte aligned, at least
  * fa_bwd_workspace_size(B,H,N,d) bytes (else FA_ERR_INVALID_ARG). Its
  * contents on entry do not matter; on exit they are scratch.
@@ -103,6 +105,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.
  */
 fa_status fa_get_device_error(void* stream);
+
+/*
+ * Measurement hook. After this call, every fa_bwd made by the calling host
+ * thread records `before` and `after` (each a cudaEvent_t passed as void*,
+ * created by the caller) on its stream immediately before and after the main
+ * backward kernel, so that kernel's own duration can be read with
+ * cudaEventElapsedTime. Pass NULL, NULL to stop. The events stay owned by the
+ * caller and must outlive the fa_bwd calls that record them. Always FA_OK.
+ */
+fa_status fa_set_bwd_main_events(void* before, void* after);
+
+/*
+ * Detail for the most recent FA_ERR_CUDA returned to the calling host thread:
+ * the cudaError_t value of the failed runtime call, -1 if a TMA descriptor
+ * could not be encoded, 0 if no CUDA failure has been returned.
+ */
+int fa_last_cuda_error(void);
 
 /* Static, NUL-terminated description of a status code. */
 const char* fa_strerror(fa_status status);

@@ -15,6 +15,9 @@ Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
   Pinned by: equality with the rows of ``attention_forward``.
 - ``attention_backward``     analytic gradients of the forward.
   Pinned by: central finite differences on N <= 16, torch fp64 autograd.
+- ``attention_backward_rows`` the work of a subset of query rows (dQ rows,
+  partial dK/dV). Pinned by: its pieces over a partition of the rows add up
+  to ``attention_backward``.
 - ``blockwise_online_softmax_attention`` the tiled merge with running max and
   running sum. Pinned by: equality with the full-row softmax on tiny inputs,
   for several block sizes.
@@ -26,6 +29,7 @@ from .attention import (  # noqa: F401
     attention_forward,
     attention_forward_rows,
     attention_backward,
+    attention_backward_rows,
     causal_visible,
 )
 from .online_softmax import blockwise_online_softmax_attention  # noqa: F401

@@ -119,22 +119,38 @@ def attention_forward_rows(q, k, v, scale: float, causal: bool, heads, rows):
     return np.stack(outs_o), np.stack(outs_l)
 
 
-def _backward_head(q, k, v, do, scale, causal):
+def _backward_head(q, k, v, do, scale, causal, rows=None):
+    """Gradients from the query rows ``rows`` (all rows if None) of one head.
+
+    dQ is returned for those rows only; dK and dV are the contributions of
+    those rows (they sum to the full dK, dV over any partition of the rows)."""
     N = q.shape[0]
-    dq = np.zeros_like(q)
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    dq = np.zeros((len(rows), q.shape[1]))
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    for c0 in range(0, N, _CHUNK):
-        r = np.arange(c0, min(N, c0 + _CHUNK))
+    for c0 in range(0, len(rows), _CHUNK):
+        r = rows[c0:c0 + _CHUNK]
         s = _scores(q[r], k, scale, r, causal)
         p, _, _ = _softmax_rows(s)          # recomputed from the definition
         dv += p.T @ do[r]                   # dV = P^T dO
         dp = do[r] @ v.T                    # dP = dO V^T
         dd = np.sum(p * dp, axis=1, keepdims=True)   # D_i = sum_j P_ij dP_ij
         ds = p * (dp - dd)                  # softmax Jacobian applied to dP
-        dq[r] = scale * (ds @ k)            # dQ = scale dS K
+        dq[c0:c0 + len(r)] = scale * (ds @ k)   # dQ = scale dS K
         dk += scale * (ds.T @ q[r])         # dK = scale dS^T Q
     return dq, dk, dv
+
+
+def attention_backward_rows(q, k, v, do, scale: float, causal: bool, heads, rows):
+    """Work of the query rows ``rows`` of the given (b, h) heads: dQ for those
+    rows [len(heads), len(rows), d], and their contributions to dK and dV
+    [len(heads), N, d]. Used to time a bounded sample of a large workload."""
+    res = [
+        _backward_head(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(do[b, h]), scale, causal, rows)
+        for (b, h) in heads
+    ]
+    return tuple(np.stack([r[i] for r in res]) for i in range(3))
 
 
 def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):

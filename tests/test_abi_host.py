@@ -14,7 +14,7 @@ FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
 def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_error",
-                          "fa_strerror", "fa_version"}
+                          "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -32,7 +32,9 @@ def test_workspace_size():
     B, H, N, d = 2, 3, 1000, 128
     rows = B * H * N
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert fa.fa_bwd_workspace_size(B, H, N, d) == up(rows * d * 4) + up(rows * 4)
+    np_ = (N + 3) // 4 * 4
+    assert fa.fa_bwd_workspace_size(B, H, N, d) == up(rows * d * 4) + 2 * up(B * H * np_ * 4)
+    assert fa.fa_bwd_workspace_size(1, 1, 17, 64) == up(17 * 64 * 4) + 2 * up(20 * 4)
     assert fa.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     assert fa.fa_bwd_workspace_size(1, 1, 1, 96) == 0
 
@@ -96,3 +98,11 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
+
+
+def test_set_bwd_main_events_is_host_only():
+    assert fa.fa_set_bwd_main_events(None, None) == fa.FA_OK
+
+
+def test_last_cuda_error_starts_clear():
+    assert fa.fa_last_cuda_error() == 0

@@ -263,3 +263,25 @@ def test_oracle_accepts_bf16_torch_inputs():
                               t.to(torch.float64).numpy(), 0.5, True)
     np.testing.assert_array_equal(o, o2)
     assert oracle.attention_forward is attention_forward
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_rows_partition_sums_to_full(causal):
+    from oracle import attention_backward_rows
+
+    B, H, n, d = 1, 2, 300, 8
+    q, k, v, do = (_rand((B, H, n, d), s) for s in (43, 44, 45, 46))
+    full = attention_backward(q, k, v, do, 0.4, causal)
+    heads = [(0, 0), (0, 1)]
+    parts = [np.arange(0, 100), np.arange(100, 257), np.arange(257, 300)]
+    dk = np.zeros((2, n, d))
+    dv = np.zeros((2, n, d))
+    for r in parts:
+        dq_r, dk_r, dv_r = attention_backward_rows(q, k, v, do, 0.4, causal, heads, r)
+        for t, (b, h) in enumerate(heads):
+            np.testing.assert_allclose(dq_r[t], full[0][b, h][r], rtol=0, atol=1e-13)
+        dk += dk_r
+        dv += dv_r
+    for t, (b, h) in enumerate(heads):
+        np.testing.assert_allclose(dk[t], full[1][b, h], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv[t], full[2][b, h], rtol=0, atol=1e-12)
