@@ -24,6 +24,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa.h")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_BF16, FA_F32 = 0, 1
+FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -33,6 +34,7 @@ _SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_set_bwd_main_events": (_I, [_P, _P]),
     "fa_last_cuda_error": (_I, []),
@@ -84,6 +86,12 @@ def fa_bwd_workspace_size(B, H, N, d) -> int:
 
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, scale, causal, stream) -> int:
     return _lib.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, scale, causal, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, stream) -> int:
+    """fa_bwd with its scratch in a fixed device array inside the library; for
+    callers that may not allocate device memory (see include/fa.h)."""
+    return _lib.fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, stream)
 
 
 def fa_get_device_error(stream) -> int:

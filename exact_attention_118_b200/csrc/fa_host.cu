@@ -209,6 +209,36 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for fa_bwd_noalloc. Some callers may not allocate device
+// memory at all: code that runs inside a host application which owns every
+// GPU allocation (a plug-in handed only its tensors), or a latency-critical
+// path where a cudaMalloc's unpredictable cost is not allowed. For them the
+// backward's workspace lives in this file-scope device array instead. Every
+// GPU that loads the library holds it (FA_NOALLOC_SCRATCH_BYTES) until exit.
+// In host code the array's name is only a stand-in, not a device address:
+// its address on each device comes from cudaGetSymbolAddress, taken once per
+// device with that device current and cached here.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch)) return cuda_fail(e);
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -298,6 +328,24 @@ fa_status fa_get_device_error(void* stream) {
     return FA_ERR_TIMEOUT;
   }
   return FA_OK;
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                         int causal, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  fa_status s = check_sizes(B, H, N, d, scale, causal);
+  if (s != FA_OK) return s;
+  if (fa::bwd_workspace_bytes(B * H, N, d) > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES))
+    return FA_ERR_UNSUPPORTED;  // the problem needs more scratch than the fixed array holds
+  if ((s = check_device()) != FA_OK) return s;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B * H, N, scale, causal, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B * H, N, scale, causal, st);
 }
 
 }  // extern "C"

@@ -100,6 +100,35 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Backward pass that allocates nothing and takes no workspace. The pages have
+ * no counterpart; this exists for callers that may not allocate device
+ * memory themselves, such as code inside a host application that owns every
+ * GPU allocation, or a latency-critical path where a cudaMalloc is not
+ * allowed. It computes exactly what fa_bwd computes, with the same arguments
+ * minus the workspace, by the same kernels.
+ *
+ * Its scratch (the dQ accumulator and two per-row arrays, as sized by
+ * fa_bwd_workspace_size) is one fixed device array inside the library of
+ * FA_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits. Problems with fa_bwd_workspace_size(B,H,N,d) >
+ * FA_NOALLOC_SCRATCH_BYTES are rejected with FA_ERR_UNSUPPORTED before any
+ * launch. No call allocates: no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture. Every call shares the one array and
+ * the array keeps the last call's contents (the call itself clears what must
+ * start at zero), so calls whose work overlaps on the GPU - on different
+ * streams, or from different threads - race on it: order them on one stream
+ * or synchronise between them.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                         float scale, int causal, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.

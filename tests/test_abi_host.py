@@ -13,7 +13,7 @@ FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
 
 def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
-    assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_error",
+    assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
     for n in names:
@@ -106,3 +106,20 @@ def test_set_bwd_main_events_is_host_only():
 
 def test_last_cuda_error_starts_clear():
     assert fa.fa_last_cuda_error() == 0
+
+
+def test_noalloc_rejects_problems_beyond_its_fixed_scratch():
+    # 32 heads x 16384 rows x d=128 needs ~269 MB of scratch: more than the array holds.
+    assert fa.fa_bwd_workspace_size(1, 32, 16384, 128) > fa.FA_NOALLOC_SCRATCH_BYTES
+    st = fa.fa_bwd_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 32, 16384, 128, 0.088, 1, None)
+    assert st == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_bwd_noalloc(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 64, 0.1, 0,
+                             None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_size_matches_header():
+    import re
+
+    with open(fa.HEADER_PATH) as f:
+        m = re.search(r"#define FA_NOALLOC_SCRATCH_BYTES \((\d+)u \* 1024u \* 1024u\)", f.read())
+    assert m and int(m.group(1)) * 1024 * 1024 == fa.FA_NOALLOC_SCRATCH_BYTES
