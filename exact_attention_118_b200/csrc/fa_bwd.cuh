@@ -21,8 +21,8 @@
 //   dV  += P^T dO_i         (TS: A = P^T bf16 in TMEM)
 //   dK  += dS^T Q_i         (TS: A = dS^T bf16 in TMEM)
 //   dQ_i^T = K_j^T dS^T     (SS: A = K_j read MN-major, B = dS from smem)
-//   dQ_i^T is drained from TMEM to shared memory and added into the fp32 dQ
-//   accumulator in global memory with one TMA reduce-add per tile.
+//   dQ_i^T is drained from TMEM by a warpgroup that stages it in shared
+//   memory and adds it into the fp32 dQ accumulator with TMA reduce-adds.
 // S and dP are double-buffered (b = iteration & 1) so the tensor core computes
 // tile i+1 while an elementwise warpgroup works on tile i; each buffer has its
 // own elementwise warpgroup, so the two groups overlap each other's waits.
@@ -125,20 +125,23 @@ struct BwdParams {
 
 template <int D>
 struct BwdLayout {
-  static constexpr int kKV = 128 * D * 2;          // K or V tile: 128 keys
-  static constexpr int kQT = 64 * D * 2;           // Q or dO tile: 64 queries
-  static constexpr int kStages = (D == 128) ? 3 : 4;  // Q/dO/lse2/D ring depth
+  static constexpr int kKV = 128 * D * 2;  // K or V tile: 128 keys
+  static constexpr int kQT = 64 * D * 2;   // Q or dO tile: 64 queries
+  static constexpr int kStages = 4;        // Q/dO/lse2/D ring depth
   static constexpr int kDSTile = 128 * 64 * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kKV;
   static constexpr int kQ = 2 * kKV;
   static constexpr int kDO = kQ + kStages * kQT;
-  static constexpr int kDS = kDO + kStages * kQT;  // [2] dS tiles [128 keys][64 queries]
-  static constexpr int kDQ = kDS + 2 * kDSTile;    // fp32 staging [64 queries][D]
-  static constexpr int kStat = kDQ + 64 * D * 4;   // [kStages] x {lse2[64], D[64]}
+  // [2] dS tiles [128 keys][64 queries]; after the dQ MMA has read tile b it
+  // doubles as the fp32 staging area for dQ_i (two halves of 32 queries).
+  static constexpr int kDS = kDO + kStages * kQT;
+  static constexpr int kStat = kDS + 2 * kDSTile;  // [kStages] x {lse2[64], D[64]}
   static constexpr int kBar = kStat + kStages * 512;
   static constexpr int kBytes = kBar + 256;
-  static constexpr int kAlloc = kBytes + 1024;
+  // The kernel checks that the dynamic shared memory base is 1 KB aligned
+  // (it is: the window starts on a 1 KB boundary) instead of reserving slack.
+  static constexpr int kAlloc = kBytes;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
@@ -166,8 +169,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int QS = L::kStages;
   constexpr int KCH = D / 64;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0u) {  // uniform over the CTA: nothing started yet
+    if (threadIdx.x == 0) atomicOr(&g_device_error, FA_DEVERR_SMEM_ALIGN);
+    return;
+  }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
@@ -179,7 +185,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_full = p_full + 2;       // [2]
   uint64_t* dq_full = ds_full + 2;      // [2]
   uint64_t* dq_empty = dq_full + 2;     // [2]
-  uint64_t* acc_full = dq_empty + 2;
+  uint64_t* stg_free = dq_empty + 2;    // [2] dS tile b free again (dQ staging read)
+  uint64_t* acc_full = stg_free + 2;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(ds_full + b, 4);
       mbar_init(dq_full + b, 1);
       mbar_init(dq_empty + b, 4);
+      mbar_init(stg_free + b, 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
@@ -237,6 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_dq);
       prefetch_tmap(&tm_lse2);
       prefetch_tmap(&tm_dsum);
       mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
@@ -363,41 +372,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float4* dd = lse2 + 16;
       const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (CAUSAL && j * 128 + 127 > q0);
       float pr[64];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sv[32];
-        tmem_ld32(tS + 32 * h, sv);
+      {
+        uint32_t sv[64];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tS + 32, sv + 32);
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = lse2[8 * h + c4];
-          const int q = 32 * h + 4 * c4;
-          pr[q + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), lam, -l4.x));
-          pr[q + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), lam, -l4.y));
-          pr[q + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), lam, -l4.z));
-          pr[q + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), lam, -l4.w));
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = lse2[c4];
+          pr[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), lam, -l4.x));
+          pr[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), lam, -l4.y));
+          pr[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), lam, -l4.z));
+          pr[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), lam, -l4.w));
         }
-        if (edge) {
+      }
+      if (edge) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int qi = q0 + 32 * h + c;
-            const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
-            if (!vis) pr[32 * h + c] = 0.f;
-          }
+        for (int c = 0; c < 64; ++c) {
+          const int qi = q0 + c;
+          const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
+          if (!vis) pr[c] = 0.f;
         }
-        uint32_t pk[16];
+      }
+      {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(pr[32 * h + 2 * c], pr[32 * h + 2 * c + 1]);
-        tmem_st16(tS + 16 * h, pk);
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+        tmem_st32(tS, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b);
 
-      // dS tile b was last read by the dQ MMA of iteration it - 2.
+      // dS tile b was last used for staging dQ of iteration it - 2.
       ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag) &&
-                                       (it < 2 || wait_parity(dq_full + b, ((it - 2) >> 1) & 1, abort_flag)));
+                                       (it < 2 || wait_parity(stg_free + b, ((it - 2) >> 1) & 1, abort_flag)));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -461,17 +471,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (wg == 1) {
     // ------------------------------------------------- dQ drain (warps 4-7)
+    // dQ_i^T sits in TMEM with the head-dim index on lanes and the 64 queries
+    // on columns. The drain copies it to the dS tile b (free once the dQ MMA
+    // that read it is done) as an fp32 [32 queries][D] half-tile, and one TMA
+    // reduce-add per half adds it into the fp32 accumulator; the TMA engine
+    // streams the reduction to L2 while the warps move on.
     setmaxnreg_dec<kRegDrain>();
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    // dQ^T rows (head-dim index) held by this thread: M = D = 128 uses every
-    // lane; M = 64 uses lanes 0-15 of each 32-lane quarter.
+    // M = D = 128 uses every lane; M = 64 uses lanes 0-15 of each quarter.
     const int drow = (D == 128) ? quarter * 32 + lane : quarter * 16 + lane;
     const bool holds = (D == 128) || (lane < 16);
-    float* stg = reinterpret_cast<float*>(smem + L::kDQ);
     const bool leader = (warp == 4 && lane == 0);
     bool ok = true;
-    // Every drain warp runs all 2*n_it named barriers, even after an abort
+    // Every drain warp runs all 4*n_it named barriers, even after an abort
     // (work is skipped instead), so no warp can be left waiting at one.
     for (int it = 0; it < n_it; ++it) {
       const int b = it & 1;
@@ -486,17 +499,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_empty + b);
       }
-      if (leader) bulk_wait_group_read0();  // previous reduce has read the staging tile
-      named_bar_sync(1, 128);
-      if (ok && holds) {
+      float* stg = reinterpret_cast<float*>(smem + L::kDS + b * L::kDSTile);
+      const int q0 = (i_start + it) * 64;
 #pragma unroll
-        for (int q = 0; q < 64; ++q) stg[q * D + drow] = __uint_as_float(v[q]);
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && leader) bulk_wait_group_read0();  // half 0 has been read
+        named_bar_sync(1, 128);
+        if (ok && holds) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) stg[q * D + drow] = __uint_as_float(v[32 * h + q]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader && ok) {
+          tma_reduce_add_3d(&tm_dq, stg, 0, q0 + 32 * h, bh);
+          bulk_commit_group();
+        }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader && ok) {
-        tma_reduce_add_3d(&tm_dq, stg, 0, (i_start + it) * 64, bh);
-        bulk_commit_group();
+      if (leader) {
+        bulk_wait_group_read0();
+        if (ok) mbar_arrive(stg_free + b);
       }
     }
     if (leader) bulk_wait_group0();

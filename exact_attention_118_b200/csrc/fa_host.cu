@@ -176,7 +176,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   fa_status s = launch_status();
   if (s != FA_OK) return s;
 
-  // 2. Main kernel. Maps: q, k, v, dO, dQ accumulator, lse2, D.
+  // 2. Main kernel. Maps: q, k, v, dO, dQ accumulator (fp32, 32-row box), lse2, D.
   alignas(64) CUtensorMap maps[7];
   if ((s = make_tmap(&maps[0], q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
@@ -186,7 +186,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   if ((s = make_tmap(&maps[3], dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
-  if ((s = make_tmap(&maps[4], dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 64,
+  if ((s = make_tmap(&maps[4], dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 32,
                      CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return s;
   if ((s = make_stat_map(&maps[5], lse2, N, Np, BH)) != FA_OK) return s;

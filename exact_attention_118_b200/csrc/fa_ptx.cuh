@@ -15,6 +15,7 @@ namespace fa {
 // The library is a single translation unit, so the word is defined here.
 __device__ unsigned int g_device_error = 0u;
 constexpr unsigned int FA_DEVERR_TIMEOUT = 1u;
+constexpr unsigned int FA_DEVERR_SMEM_ALIGN = 2u;  // dynamic shared memory not 1 KB aligned
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -119,7 +120,8 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_
                : "memory");
 }
 
-// Element-wise fp32 add of a shared-memory tile into global memory.
+// Element-wise fp32 add of a shared-memory tile into global memory (the
+// reduction happens in L2; the TMA engine streams it in the background).
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, const void* smem_src, int c0, int c1,
                                                   int c2) {
   asm volatile(
