@@ -27,8 +27,8 @@
 // tile i+1 while an elementwise warpgroup works on tile i; each buffer has its
 // own elementwise warpgroup, so the two groups overlap each other's waits.
 //
-// Roles (512 threads): warp 0 TMA producer (Q, dO, lse2 and D tiles), warp 1
-// MMA issuer, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
+// Roles (512 threads): warp 0 TMA producer (Q, dO, lse2 and D tiles), warps 1
+// and 2 MMA issuers, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
 // dQ^T), warps 8-11 and 12-15 two elementwise warpgroups (thread = key row)
 // that take alternate query tiles.
 #pragma once
@@ -145,8 +145,8 @@ struct BwdLayout {
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-// Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warp 1
-// MMA issuer and TMEM owner, warps 2-3 idle), 4-7 dQ drain, 8-11 elementwise
+// Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warps 1
+// and 2 MMA issuers, warp 1 also TMEM owner, warp 3 idle), 4-7 dQ drain, 8-11 elementwise
 // (even iterations, TMEM buffer 0), 12-15 elementwise (odd iterations, buffer
 // 1). Launched at 128 registers per thread (512 x 128 = the 64K register
 // file; each SM sub-partition holds one warp of every warpgroup); the groups
@@ -186,7 +186,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* dq_full = ds_full + 2;      // [2]
   uint64_t* dq_empty = dq_full + 2;     // [2]
   uint64_t* stg_free = dq_empty + 2;    // [2] dS tile b free again (dQ staging read)
-  uint64_t* acc_full = stg_free + 2;
+  uint64_t* y_done = stg_free + 2;      // [2] dV/dK of the buffer's last iteration done
+  uint64_t* acc_full = y_done + 2;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < QS; ++s) {
       mbar_init(qd_full + s, 1);
-      mbar_init(qd_empty + s, 1);
+      mbar_init(qd_empty + s, 2);  // one release per MMA issuer
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
@@ -221,9 +222,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(dq_full + b, 1);
       mbar_init(dq_empty + b, 4);
       mbar_init(stg_free + b, 1);
+      mbar_init(y_done + b, 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -271,9 +273,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_parity_drain(kv_full, 0);
       for (int it = max(0, issued - QS); it < issued; ++it) wait_parity_drain(qd_full + it % QS, (it / QS) & 1);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------- MMA issuers
+    // One issuing thread cannot keep the tensor core busy with these MMA
+    // shapes, so two share the work: X (warp 1) issues S^T and dQ^T, Y (warp
+    // 2) issues dP^T, dV and dK. They meet at TMEM buffer S[b]: S^T(it+2) may
+    // overwrite it only after Y's dV(it)/dK(it) have read P^T/dS^T from it
+    // (barrier y_done[b]). Both read the Q/dO stage, so qd_empty takes one
+    // release from each.
     if (lane == 0) {
+      const bool is_x = (warp == 1);
       constexpr uint32_t kIdST = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T: K-major A and B
       constexpr uint32_t kIdAcc = idesc_bf16(128, D, 0, 1);  // dV, dK: A TMEM, B MN-major
       constexpr uint32_t kIdDQ = idesc_bf16(D, 64, 1, 1);    // dQ^T: A, B MN-major
@@ -310,38 +319,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = wait_parity(kv_full, 0, abort_flag) && wait_parity(qd_full, 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_t(0, k_addr, q_addr);
-        mma_commit(s_full + 0);
-        issue_t(128, v_addr, do_addr);
-        mma_commit(dp_full + 0);
+        if (is_x) {
+          issue_t(0, k_addr, q_addr);
+          mma_commit(s_full + 0);
+          mma_commit(qd_empty + 0);
+        } else {
+          issue_t(128, v_addr, do_addr);
+          mma_commit(dp_full + 0);
+        }
       }
       for (int it = 0; ok && it < n_it; ++it) {
         const int b = it & 1, s = it % QS;
         const int nb = b ^ 1, ns = (it + 1) % QS;
         const bool has_next = it + 1 < n_it;
-        if (has_next) {
-          if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
+        if (is_x) {
+          if (has_next) {
+            if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
+            if (it >= 1 && !(ok = wait_parity(y_done + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_t(64 * nb, k_addr, q_addr + ns * L::kQT);
+            mma_commit(s_full + nb);
+            mma_commit(qd_empty + ns);
+          }
+          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_t(64 * nb, k_addr, q_addr + ns * L::kQT);
-          mma_commit(s_full + nb);
-        }
-        if (!(ok = wait_parity(p_full + b, (it >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_acc(t_dv, 64 * b, do_addr + s * L::kQT, it > 0);
-        if (has_next) {
-          if (it >= 1 && !(ok = wait_parity(dq_empty + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
+          issue_dq(b);
+          mma_commit(dq_full + b);
+        } else {
+          if (!(ok = wait_parity(p_full + b, (it >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_t(128 + 64 * nb, v_addr, do_addr + ns * L::kQT);
-          mma_commit(dp_full + nb);
+          issue_acc(t_dv, 64 * b, do_addr + s * L::kQT, it > 0);
+          if (has_next) {
+            if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
+            if (it >= 1 && !(ok = wait_parity(dq_empty + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_t(128 + 64 * nb, v_addr, do_addr + ns * L::kQT);
+            mma_commit(dp_full + nb);
+          }
+          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_acc(t_dk, 64 * b + 32, q_addr + s * L::kQT, it > 0);
+          mma_commit(y_done + b);
+          mma_commit(qd_empty + s);
         }
-        if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_acc(t_dk, 64 * b + 32, q_addr + s * L::kQT, it > 0);
-        issue_dq(b);
-        mma_commit(dq_full + b);
-        mma_commit(qd_empty + s);
       }
-      if (ok) mma_commit(acc_full);
+      if (ok && !is_x) mma_commit(acc_full);
+      // Let every MMA both issuers started finish before TMEM is freed.
       mma_commit(mma_done);
       wait_parity_drain(mma_done, 0);
     }
