@@ -410,6 +410,28 @@ def run_native(args):
     return 0
 
 
+def run_profile_case(args):
+    """Untimed forward+backward launches for an ncu capture: B=1, N=16384,
+    d=128, `--profile-case` heads, non-causal (or causal with --causal), three
+    passes. Prints nothing but "ok"."""
+    import torch
+
+    import exact_attention_118_b200 as fa
+
+    h = args.profile_case
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    q, k, v, do = (torch.randn(B, h, N, D, device="cuda", generator=g).to(torch.bfloat16) for _ in range(4))
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, h, N, D), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        o, lse = fa.attention_forward(q, k, v, causal=args.causal)
+        fa.attention_backward(q, k, v, o, lse, do, causal=args.causal, workspace=ws)
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    print("ok")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,7 +439,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", type=int, default=0, metavar="HEADS",
+                    help="run untimed fwd+bwd launches with this many heads (for ncu) and exit")
+    ap.add_argument("--causal", action="store_true", help="with --profile-case: causal mask")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case(args)
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     if args.impl == "reference":

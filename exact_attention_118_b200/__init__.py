@@ -2,7 +2,7 @@
 
 The functions ``fa_fwd``, ``fa_bwd``, ``fa_bwd_workspace_size``,
 ``fa_get_device_error``, ``fa_set_bwd_main_events``, ``fa_last_cuda_error``,
-``fa_strerror`` and ``fa_version`` have the names and
+``fa_selftest_wait_timeout``, ``fa_strerror`` and ``fa_version`` have the names and
 arguments of the C ABI in ``include/fa.h`` (pointers and the stream are plain
 integers) and only marshal arguments. ``attention_forward`` and
 ``attention_backward`` are conveniences that take torch CUDA tensors, allocate
@@ -38,6 +38,7 @@ _SIGNATURES = {
     "fa_get_device_error": (_I, [_P]),
     "fa_set_bwd_main_events": (_I, [_P, _P]),
     "fa_last_cuda_error": (_I, []),
+    "fa_selftest_wait_timeout": (_I, [_P]),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -104,6 +105,10 @@ def fa_set_bwd_main_events(before, after) -> int:
 
 def fa_last_cuda_error() -> int:
     return _lib.fa_last_cuda_error()
+
+
+def fa_selftest_wait_timeout(stream) -> int:
+    return _lib.fa_selftest_wait_timeout(stream)
 
 
 def fa_strerror(status: int) -> str:

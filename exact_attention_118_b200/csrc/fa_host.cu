@@ -209,6 +209,21 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   return launch_status();
 }
 
+// Failure-detection self-test: one thread waits, through the same bounded
+// wait the kernels use, on an mbarrier that nothing ever completes. The wait
+// gives up after its time limit, records FA_DEVERR_TIMEOUT in the device error
+// word and the kernel returns normally.
+__global__ void fa_selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    fa::fence_barrier_init();
+    fa::wait_parity(&bar, 0, &abort_flag);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Fixed scratch for fa_bwd_noalloc. Some callers may not allocate device
 // memory at all: code that runs inside a host application which owns every
@@ -310,6 +325,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 }
 
 int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+fa_status fa_selftest_wait_timeout(void* stream) {
+  fa_status s = check_device();
+  if (s != FA_OK) return s;
+  fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
+}
 
 fa_status fa_set_bwd_main_events(void* before, void* after) {
   t_bwd_ev_before = static_cast<cudaEvent_t>(before);

@@ -152,6 +152,17 @@ fa_status fa_set_bwd_main_events(void* before, void* after);
  */
 int fa_last_cuda_error(void);
 
+/*
+ * Test hook for the failure-detection path. Launches one thread on `stream`
+ * that waits, through the same bounded wait every kernel of this library
+ * uses, on a barrier nothing ever completes. After the wait's time limit
+ * (about 2 s) it gives up, records the timeout in the device error word and
+ * the kernel exits normally, so the next fa_get_device_error(stream) returns
+ * FA_ERR_TIMEOUT and the context stays usable. No GPU fault is involved.
+ * Returns FA_OK once launched.
+ */
+fa_status fa_selftest_wait_timeout(void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_strerror(fa_status status);
 

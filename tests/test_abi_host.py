@@ -14,7 +14,8 @@ FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
 def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
-                          "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_strerror", "fa_version"}
+                          "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
+                          "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
