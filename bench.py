@@ -42,10 +42,13 @@ B, H, N, D = 1, 16, 16384, 128
 SEED = 3
 WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then causal"
 
-# DRAM traffic of the main backward kernel, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum per launch, non-causal launch
-# of the workload above). Valid only for the kernel source it was taken on.
-BWD_TRAFFIC = {"bytes": None, "source_sha256": None, "profile": None}
+# DRAM traffic of one non-causal main backward launch of the workload above:
+# dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the same
+# kernel at H=4 (124.7 MB), scaled by the number of heads (traffic grows with
+# the heads processed). Valid only for the kernel source it was taken on.
+BWD_TRAFFIC = {"bytes": 4 * 124.686592e6,
+               "source_sha256": "45105d16dd5f6e9d5b2a0caa40252317694ff516b61b1b53c10eec4b1ce10159",
+               "profile": "profiles/fa_bwd_kernel_b1h4_n16384_d128.md"}
 
 
 def _flops(causal: bool):
@@ -119,6 +122,28 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# ------------------------------------------------------------ rank helpers
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the default process group (identity when
+    there is none or it has one rank). Used for the timed region."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(step_flops: float, world: int, ms_total_max: float, steps: int):
+    """(ms per step, whole-job TFLOP/s): every rank runs its own replica, so
+    the job's FLOPs are world * step_flops per step, over the slowest rank."""
+    ms_per_step = ms_total_max / steps
+    return ms_per_step, step_flops * world / (ms_per_step / 1e3) / 1e12
 
 
 # ------------------------------------------------------------ oracle sample
@@ -211,13 +236,6 @@ def run_native(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # CPU baseline first (rank 0, one GPU only), before the GPU is busy.
     cpu_baseline = None
     x_cpu = make_inputs(B, H, N, D, SEED)
@@ -306,9 +324,8 @@ def run_native(args):
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     check(fa.fa_get_device_error(sp), "timed region")
-    ms_total = max_over_ranks(start.elapsed_time(stop))
-    ms_per_step = ms_total / args.steps
-    value = step_flops * world / (ms_per_step / 1e3) / 1e12
+    ms_total = max_over_ranks(start.elapsed_time(stop), dev)
+    ms_per_step, value = aggregate(step_flops, world, ms_total, args.steps)
 
     # per-pass breakdown (events around each call) and the main backward kernel
     def med(xs):
@@ -346,15 +363,17 @@ def run_native(args):
                                 "frac_of_peak": fb / per[c]["bwd_ms"] / 1e9 / peak,
                                 "main_kernel_ms": per[c]["bwd_main_ms"]}
 
-    # Roofline of the dominant kernel: the main backward kernel (both masks).
-    main_total_ms = sum(bwd_main_ms[False]) + sum(bwd_main_ms[True])
-    main_flops = args.steps * (bwd_nc + bwd_c)
-    achieved = main_flops / (main_total_ms / 1e3) / 1e12
+    # Roofline of the dominant kernel: the main backward kernel, non-causal
+    # launch (the largest share of the step), from its own CUDA events.
+    main_ms = statistics.mean(bwd_main_ms[False])
+    achieved = bwd_nc / (main_ms / 1e3) / 1e12
     traffic = None
     if BWD_TRAFFIC["bytes"] is not None and BWD_TRAFFIC["source_sha256"] == _bwd_source_sha():
         traffic = BWD_TRAFFIC["bytes"]
-    roofline = {"kernel": "fa_bwd_kernel<128> (main backward)", "bound": "tensor", "achieved": achieved,
-                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+    roofline = {"kernel": "fa_bwd_kernel<128, non-causal> (main backward)", "bound": "tensor",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic, "traffic_source": BWD_TRAFFIC["profile"] if traffic else None,
+                "algorithmic_flops_per_launch": bwd_nc, "avg_launch_ms": main_ms,
                 "peak_kind": f"{peak_kind} bf16 dense (burst); sustained {peak_sus}",
                 "frac_of_sustained": achieved / peak_sus}
 
@@ -383,7 +402,7 @@ def run_native(args):
     b_.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(a.elapsed_time(b_)) / e2e_steps
+    e2e_ms = max_over_ranks(a.elapsed_time(b_), dev) / e2e_steps
     check(fa.fa_get_device_error(sp), "e2e")
 
     line = {
