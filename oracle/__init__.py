@@ -18,6 +18,10 @@ Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
 - ``attention_backward_rows`` the work of a subset of query rows (dQ rows,
   partial dK/dV). Pinned by: its pieces over a partition of the rows add up
   to ``attention_backward``.
+- ``attention_forward_gqa`` / ``attention_backward_gqa`` grouped K/V heads
+  (MQA/GQA): the definition with K/V heads repeated per group; dK, dV summed
+  over the group. Pinned by: central finite differences with respect to the
+  shared K/V tensors, the MQA closed form for Q = 0, and group size 1 = MHA.
 - ``blockwise_online_softmax_attention`` the tiled merge with running max and
   running sum. Pinned by: equality with the full-row softmax on tiny inputs,
   for several block sizes.
@@ -30,6 +34,8 @@ from .attention import (  # noqa: F401
     attention_forward_rows,
     attention_backward,
     attention_backward_rows,
+    attention_backward_gqa,
+    attention_forward_gqa,
     causal_visible,
 )
 from .online_softmax import blockwise_online_softmax_attention  # noqa: F401

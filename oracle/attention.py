@@ -172,3 +172,33 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
         for h in range(H):
             dq[b, h], dk[b, h], dv[b, h] = _backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal)
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- grouped K/V
+# Multi-query / grouped-query attention: several query heads share one K/V
+# head ("FlashAttention原理：从原始Attention到FlashAttention", blog.csdn.net,
+# related-article notes on MQA/GQA: in MQA the query keeps all its heads while
+# key and value keep a single shared head). Query head h of H reads K/V head
+# h // (H // H_kv). The definition is standard attention with every K/V head
+# repeated for its group; the gradient of a shared K/V head is the sum of the
+# gradients its group's query heads send it.
+
+def _repeat_kv(x, group: int) -> np.ndarray:
+    return np.repeat(_f64(x), group, axis=1)
+
+
+def attention_forward_gqa(q, k, v, scale: float, causal: bool):
+    """q [B, H, N, d]; k, v [B, H_kv, N, d] with H % H_kv == 0."""
+    H, Hkv = q.shape[1], k.shape[1]
+    assert H % Hkv == 0
+    g = H // Hkv
+    return attention_forward(q, _repeat_kv(k, g), _repeat_kv(v, g), scale, causal)
+
+
+def attention_backward_gqa(q, k, v, do, scale: float, causal: bool):
+    """dQ [B, H, N, d]; dK, dV [B, H_kv, N, d] (summed over each group)."""
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    g = H // Hkv
+    dq, dk, dv = attention_backward(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal)
+    return dq, dk.reshape(B, Hkv, g, N, -1).sum(axis=2), dv.reshape(B, Hkv, g, N, -1).sum(axis=2)

@@ -285,3 +285,55 @@ def test_backward_rows_partition_sums_to_full(causal):
     for t, (b, h) in enumerate(heads):
         np.testing.assert_allclose(dk[t], full[1][b, h], rtol=0, atol=1e-12)
         np.testing.assert_allclose(dv[t], full[2][b, h], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ grouped K/V heads
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_finite_differences_on_shared_kv(causal):
+    from oracle import attention_backward_gqa, attention_forward_gqa
+
+    B, H, Hkv, n, d, h = 1, 4, 2, 7, 3, 1e-6
+    q, do = _rand((B, H, n, d), 50), _rand((B, H, n, d), 51)
+    k, v = _rand((B, Hkv, n, d), 52), _rand((B, Hkv, n, d), 53)
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward_gqa(q_, k_, v_, 0.7, causal)
+        return float(np.sum(o * do))
+
+    grads = attention_backward_gqa(q, k, v, do, 0.7, causal)
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            ap, am = [q.copy(), k.copy(), v.copy()], [q.copy(), k.copy(), v.copy()]
+            ap[which][idx] += h
+            am[which][idx] -= h
+            num[idx] = (loss(*ap) - loss(*am)) / (2 * h)
+        assert np.max(np.abs(num - g)) <= 1e-6 * max(1.0, np.max(np.abs(g))), which
+
+
+def test_mqa_zero_query_closed_form():
+    # One shared K/V head, Q = 0: every query head averages the shared V
+    # over its visible keys (prefix mean under the causal mask).
+    from oracle import attention_forward_gqa
+
+    B, H, n, d = 1, 3, 9, 2
+    q = np.zeros((B, H, n, d))
+    k, v = _rand((B, 1, n, d), 54), _rand((B, 1, n, d), 55)
+    o, lse = attention_forward_gqa(q, k, v, 1.0, True)
+    prefix_mean = np.cumsum(v[0, 0], axis=0) / (np.arange(n) + 1)[:, None]
+    for hh in range(H):
+        np.testing.assert_allclose(o[0, hh], prefix_mean, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[0, hh], np.log(np.arange(n) + 1), rtol=0, atol=1e-14)
+
+
+def test_gqa_group_size_one_is_mha():
+    from oracle import attention_backward_gqa, attention_forward_gqa
+
+    q, k, v, do = (_rand((2, 3, 11, 4), s) for s in (56, 57, 58, 59))
+    o1, l1 = attention_forward_gqa(q, k, v, 0.5, True)
+    o2, l2 = attention_forward(q, k, v, 0.5, True)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    for a, b in zip(attention_backward_gqa(q, k, v, do, 0.5, True), attention_backward(q, k, v, do, 0.5, True)):
+        np.testing.assert_array_equal(a, b)
