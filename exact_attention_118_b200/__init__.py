@@ -34,6 +34,9 @@ _SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_gqa_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_set_bwd_main_events": (_I, [_P, _P]),
@@ -89,6 +92,19 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, sca
     return _lib.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, scale, causal, stream)
 
 
+def fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) -> int:
+    return _lib.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
+
+
+def fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, o_dtype, stream) -> int:
+    return _lib.fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, o_dtype, stream)
+
+
+def fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, d, scale, causal, stream) -> int:
+    return _lib.fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, d, scale, causal,
+                           stream)
+
+
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, stream) -> int:
     """fa_bwd with its scratch in a fixed device array inside the library; for
     callers that may not allocate device memory (see include/fa.h)."""
@@ -137,43 +153,52 @@ def _shape(q):
 
 
 def attention_forward(q, k, v, scale=None, causal=False, out_fp32=False, out=None, lse=None):
-    """O, lse = attention(q, k, v) on the GPU. q, k, v: contiguous bf16 CUDA
-    tensors [B, H, N, d]. Returns (O [B,H,N,d] bf16 or fp32, lse [B,H,N] fp32)."""
+    """O, lse = attention(q, k, v) on the GPU. q: contiguous bf16 CUDA tensor
+    [B, H, N, d]; k, v: [B, Hkv, N, d] with H % Hkv == 0 (Hkv = H for
+    multi-head attention). Returns (O [B,H,N,d] bf16 or fp32, lse [B,H,N] fp32)."""
     import torch
 
     B, H, N, d = _shape(q)
+    Hkv = int(k.shape[1]) if k.dim() == 4 else -1
     if scale is None:
         scale = d ** -0.5
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
-            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of equal shape")
+    for t, heads in ((q, H), (k, Hkv), (v, Hkv)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, heads, N, d):
+            raise ValueError("q [B,H,N,d] and k, v [B,Hkv,N,d] must be contiguous bf16 CUDA tensors")
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, N, d,
-                float(scale), int(bool(causal)), FA_F32 if out.dtype == torch.float32 else FA_BF16,
-                _stream_ptr(torch, q.device))
+    st = fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Hkv, N, d,
+                    float(scale), int(bool(causal)), FA_F32 if out.dtype == torch.float32 else FA_BF16,
+                    _stream_ptr(torch, q.device))
     _check(st, "fa_fwd")
     return out, lse
 
 
 def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None):
-    """dQ, dK, dV of attention on the GPU, all bf16 [B, H, N, d]."""
+    """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of attention on the GPU, all bf16."""
     import torch
 
     B, H, N, d = _shape(q)
+    Hkv = int(k.shape[1]) if k.dim() == 4 else -1
     if scale is None:
         scale = d ** -0.5
+    for t, shape in ((q, (B, H, N, d)), (k, (B, Hkv, N, d)), (v, (B, Hkv, N, d)), (o, (B, H, N, d)),
+                     (do, (B, H, N, d))):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError("q, o, dO [B,H,N,d] and k, v [B,Hkv,N,d] must be contiguous bf16 CUDA tensors")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, N]")
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    ws_bytes = fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                B, H, N, d, float(scale), int(bool(causal)), _stream_ptr(torch, q.device))
+    st = fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                    B, H, Hkv, N, d, float(scale), int(bool(causal)), _stream_ptr(torch, q.device))
     _check(st, "fa_bwd")
     return dq, dk, dv
 

@@ -10,9 +10,10 @@
 //   D_i = rowsum(dO_i * O_i),    dS = P * (dP - D),
 //   dQ = scale * dS K,           dK = scale * dS^T Q.
 //
-// Main kernel: one CTA per (batch*head, 128-key tile j); it loops over
+// Main kernel: one CTA per (batch*K/V head, 128-key tile j); it loops over
 // 64-query tiles i (causal: only i with a visible query, the masked upper
-// triangle is skipped) and keeps dK_j, dV_j accumulating in TMEM. Everything is
+// triangle is skipped) of every query head reading that K/V head, and keeps
+// dK_j, dV_j accumulating in TMEM. Everything is
 // computed transposed (keys on TMEM lanes) so P^T and dS^T can feed the dV/dK
 // MMAs straight from TMEM:
 //   S^T  = K_j Q_i^T        (SS, M=128 keys, N=64 queries)   -> TMEM S[b]
@@ -52,17 +53,28 @@ inline size_t bwd_workspace_bytes(int BH, int N, int d) {
   return align256(rows * d * sizeof(float)) + 2 * align256(srows * sizeof(float));
 }
 
+// Grouped-query attention (Hkv < H) appends fp32 dK and dV accumulators
+// [2][B*Hkv*N*d], for when a K/V head's query heads are split across CTAs.
+inline size_t bwd_kv_acc_bytes(int B, int Hkv, int N, int d) {
+  return align256(static_cast<size_t>(B) * Hkv * N * d * sizeof(float));
+}
+inline size_t bwd_gqa_workspace_bytes(int B, int H, int Hkv, int N, int d) {
+  return bwd_workspace_bytes(B * H, N, d) + (Hkv < H ? 2 * bwd_kv_acc_bytes(B, Hkv, N, d) : 0);
+}
+
 // ------------------------------------------------- D = rowsum(dO*O), lse2
 // For every query row: D = sum_k dO_k * O_k, lse2 = lse * log2(e) (the
 // forward's natural-log normaliser moved to base 2 for the exp2 recompute),
 // both written with the padded row stride Np; and the row of the fp32 dQ
-// accumulator is zeroed (same rows, same pass).
+// accumulator is zeroed (same rows, same pass). kv_n4 float4s at kv_acc (the
+// split grouped-query dK/dV accumulators, or none) are zeroed too.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse, float* __restrict__ lse2,
                                                          float* __restrict__ dsum, float* __restrict__ dq_acc,
-                                                         long long rows, int N, int Np) {
+                                                         long long rows, int N, int Np, float* __restrict__ kv_acc,
+                                                         long long kv_n4) {
   constexpr int TPR = D / 8;  // threads per row, 16 bytes of each tensor per thread
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int part = static_cast<int>(tid % TPR);
@@ -93,6 +105,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  const long long all = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = tid; i < kv_n4; i += all)
+    reinterpret_cast<float4*>(kv_acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // --------------------------------------------------------- dQ fp32 -> bf16
@@ -113,9 +128,14 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
 
 // ------------------------------------------------------------------ main kernel
 struct BwdParams {
-  void* dk;  // bf16 [BH, N, D]
-  void* dv;  // bf16 [BH, N, D]
-  int BH;
+  void* dk;       // bf16 [B, Hkv, N, D]      (n_split == 1)
+  void* dv;       // bf16 [B, Hkv, N, D]      (n_split == 1)
+  float* dk_acc;  // fp32 [B, Hkv, N, D], zeroed (n_split > 1)
+  float* dv_acc;  // fp32 [B, Hkv, N, D], zeroed (n_split > 1)
+  int BH;         // batch * K/V heads * n_split: one CTA per (unit, 128-key tile)
+  int H;          // query heads
+  int Hkv;        // K/V heads; query heads [g*H/Hkv, (g+1)*H/Hkv) share K/V head g
+  int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv)
   int N;
   int n_kv;          // ceil(N / 128)
   int n_q;           // ceil(N / 64)
@@ -197,16 +217,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int N = p.N;
 
   // Causal: key tile 0 sees every query tile, so low j first (heaviest).
-  int j, bh;
+  int j, unit;
   if (CAUSAL) {
     j = static_cast<int>(blockIdx.x) / p.BH;
-    bh = static_cast<int>(blockIdx.x) % p.BH;
+    unit = static_cast<int>(blockIdx.x) % p.BH;
   } else {
-    bh = static_cast<int>(blockIdx.x) / p.n_kv;
+    unit = static_cast<int>(blockIdx.x) / p.n_kv;
     j = static_cast<int>(blockIdx.x) % p.n_kv;
   }
+  // The CTA walks every query tile of its share of the query heads that read
+  // K/V head bkv (the one head, for multi-head attention): dK and dV
+  // accumulate on chip over that share, and across the n_split shares in
+  // fp32 global memory.
+  const int bkv = unit / p.n_split;
+  const int group = p.H / p.Hkv / p.n_split;  // query heads of this CTA
+  const int qh0 = (bkv / p.Hkv) * p.H + (bkv % p.Hkv) * (p.H / p.Hkv) + (unit % p.n_split) * group;
   const int i_start = CAUSAL ? 2 * j : 0;  // first 64-query tile with a visible query
-  const int n_it = p.n_q - i_start;        // >= 1 since 128*j < N
+  const int n_iq = p.n_q - i_start;        // query tiles per head (>= 1 since 128*j < N)
+  const int n_it = group * n_iq;
+  auto q_start = [&](int it) { return (i_start + it % n_iq) * 64; };
+  auto q_head = [&](int it) { return qh0 + it / n_iq; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -252,22 +282,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_dsum);
       mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
       for (int c = 0; c < KCH; ++c) {
-        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, j * 128, bh);
-        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, j * 128, bh);
+        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, j * 128, bkv);
+        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, j * 128, bkv);
       }
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
         const int s = it % QS, u = it / QS;
         if (it >= QS && !wait_parity(qd_empty + s, (u - 1) & 1, abort_flag)) break;
-        const int q0 = (i_start + it) * 64;
+        const int q0 = q_start(it), bhq = q_head(it);
         uint8_t* st = smem + L::kStat + s * 512;
         mbar_arrive_expect_tx(qd_full + s, kStageTx);
         for (int c = 0; c < KCH; ++c) {
-          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, q0, bh);
-          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, q0, bh);
+          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, q0, bhq);
+          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, q0, bhq);
         }
-        tma_load_2d(st, &tm_lse2, qd_full + s, q0, bh);
-        tma_load_2d(st + 256, &tm_dsum, qd_full + s, q0, bh);
+        tma_load_2d(st, &tm_lse2, qd_full + s, q0, bhq);
+        tma_load_2d(st + 256, &tm_dsum, qd_full + s, q0, bhq);
         issued = it + 1;
       }
       wait_parity_drain(kv_full, 0);
@@ -386,7 +416,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int it = e; it < n_it; it += 2) {
       const int s = it % QS;
-      const int q0 = (i_start + it) * 64;
+      const int q0 = q_start(it);
       ok = __all_sync(0xffffffffu, wait_parity(qd_full + s, (it / QS) & 1, abort_flag) &&
                                        wait_parity(s_full + b, (it >> 1) & 1, abort_flag));
       if (!ok) break;
@@ -472,15 +502,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ok) {
         tc_fence_after();
         const bool valid = kj < N;
-        const size_t row = static_cast<size_t>(bh) * N + (valid ? kj : 0);
+        const size_t row = static_cast<size_t>(bkv) * N + (valid ? kj : 0);
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e ? p.dk : p.dv) + row * D;
+        float* acc = (e ? p.dk_acc : p.dv_acc) + row * D;
         const uint32_t col = e ? t_dk : t_dv;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_off + col + c, v);
           tmem_wait_ld();
-          if (valid) {
+          if (valid && p.n_split > 1) {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              red_add_v4(acc + c + 4 * x, __uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                         __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+          } else if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -523,7 +559,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) mbar_arrive(dq_empty + b);
       }
       float* stg = reinterpret_cast<float*>(smem + L::kDS + b * L::kDSTile);
-      const int q0 = (i_start + it) * 64;
+      const int q0 = q_start(it), bhq = q_head(it);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (h == 1 && leader) bulk_wait_group_read0();  // half 0 has been read
@@ -535,7 +571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (leader && ok) {
-          tma_reduce_add_3d(&tm_dq, stg, 0, q0 + 32 * h, bh);
+          tma_reduce_add_3d(&tm_dq, stg, 0, q0 + 32 * h, bhq);
           bulk_commit_group();
         }
       }

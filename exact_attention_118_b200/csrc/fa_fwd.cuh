@@ -37,7 +37,9 @@ namespace fa {
 struct FwdParams {
   void* o;
   float* lse;
-  int BH;
+  int BH;   // batch * query heads
+  int H;    // query heads
+  int Hkv;  // K/V heads (H % Hkv == 0; query head h reads K/V head h / (H / Hkv))
   int N;
   int n_pairs;       // ceil(N / 256): CTAs per (batch, head)
   float scale_log2;  // scale * log2(e)
@@ -134,6 +136,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // K/V head of this query head (grouped-query attention; equal for MHA).
+      const int bkv = (bh / p.H) * p.Hkv + (bh % p.H) / (p.H / p.Hkv);
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -147,12 +151,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(k_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, j * 128, bh);
+          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, j * 128, bkv);
         k_issued = j + 1;
         if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, j * 128, bh);
+          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, j * 128, bkv);
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.

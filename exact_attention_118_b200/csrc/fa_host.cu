@@ -157,10 +157,31 @@ fa_status launch_bwd_main(const CUtensorMap* maps, const fa::BwdParams& p, cudaS
   return s;
 }
 
+// How many CTAs share one K/V head's query heads in the backward (a divisor
+// of the group size H / Hkv; 1 for multi-head attention). One CTA per
+// (K/V head, key tile) keeps dK and dV on chip for the whole group, but a few
+// K/V heads give too few CTAs to fill the GPU, and causal key tiles differ
+// in cost. So take the smallest divisor that gives at least 8 CTAs per SM
+// (the whole group when none does); shares then add their partial dK and dV
+// in fp32 global memory.
+int bwd_split(int B, int H, int Hkv, int N) {
+  const int group = H / Hkv;
+  if (group == 1) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+    sms = 148;
+  const long long base = static_cast<long long>((N + 127) / 128) * B * Hkv;
+  for (int s = 1; s < group; ++s)
+    if (group % s == 0 && base * s >= 8LL * sms) return s;
+  return group;
+}
+
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                     void* dq, void* dk, void* dv, void* workspace, int BH, int N, float scale, int causal,
-                     cudaStream_t st) {
+                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv, int N, float scale,
+                     int causal, cudaStream_t st) {
+  const int BH = B * H, BHkv = B * Hkv;
   const long long rows = static_cast<long long>(BH) * N;
   const int Np = fa::stat_stride(N);
   char* ws = static_cast<char*>(workspace);
@@ -168,11 +189,19 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   float* lse2 = reinterpret_cast<float*>(ws + fa::align256(rows * D * sizeof(float)));
   float* dsum = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) +
                                          fa::align256(static_cast<size_t>(BH) * Np * sizeof(float)));
+  const int n_split = bwd_split(B, H, Hkv, N);
+  float* dk_acc = nullptr;
+  float* dv_acc = nullptr;
+  const long long kv_elems = static_cast<long long>(BHkv) * N * D;
+  if (n_split > 1) {
+    dk_acc = reinterpret_cast<float*>(ws + fa::bwd_workspace_bytes(BH, N, D));
+    dv_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(dk_acc) + fa::bwd_kv_acc_bytes(B, Hkv, N, D));
+  }
 
-  // 1. D = rowsum(dO * O), lse2 = lse * log2(e), dQ accumulator = 0.
+  // 1. D = rowsum(dO * O), lse2 = lse * log2(e), dQ (and split dK/dV) accumulators = 0.
   fa::fa_bwd_dot_kernel<D><<<helper_grid(rows * (D / 8)), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dsum, dq_acc, rows,
-      N, Np);
+      N, Np, dk_acc, n_split > 1 ? (2 * fa::bwd_kv_acc_bytes(B, Hkv, N, D)) / 16 : 0);
   fa_status s = launch_status();
   if (s != FA_OK) return s;
 
@@ -181,8 +210,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   if ((s = make_tmap(&maps[0], q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
-  if ((s = make_bf16_tile_map(&maps[1], k, D, N, BH)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&maps[2], v, D, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&maps[1], k, D, N, BHkv)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&maps[2], v, D, N, BHkv)) != FA_OK) return s;
   if ((s = make_tmap(&maps[3], dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
@@ -194,7 +223,12 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   fa::BwdParams p;
   p.dk = dk;
   p.dv = dv;
-  p.BH = BH;
+  p.dk_acc = dk_acc;
+  p.dv_acc = dv_acc;
+  p.BH = BHkv * n_split;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.n_split = n_split;
   p.N = N;
   p.n_kv = (N + 127) / 128;
   p.n_q = (N + 63) / 64;
@@ -206,6 +240,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   // 3. dq = bf16(dQ accumulator).
   const long long n8 = rows * D / 8;
   fa::fa_bwd_dq_convert_kernel<<<helper_grid(n8), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  if ((s = launch_status()) != FA_OK || n_split == 1) return s;
+
+  // 4. Split grouped-query heads: dk, dv = bf16(their fp32 accumulators).
+  fa::fa_bwd_dq_convert_kernel<<<helper_grid(kv_elems / 8), 256, 0, st>>>(
+      dk_acc, static_cast<__nv_bfloat16*>(dk), kv_elems / 8);
+  if ((s = launch_status()) != FA_OK) return s;
+  fa::fa_bwd_dq_convert_kernel<<<helper_grid(kv_elems / 8), 256, 0, st>>>(
+      dv_acc, static_cast<__nv_bfloat16*>(dv), kv_elems / 8);
   return launch_status();
 }
 
@@ -271,25 +313,28 @@ const char* fa_strerror(fa_status s) {
   return "unknown status";
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                 float scale, int causal, fa_dtype o_dtype, void* stream) {
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                     int N, int d, float scale, int causal, fa_dtype o_dtype, void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
   if (o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
   fa_status s = check_sizes(B, H, N, d, scale, causal);
   if (s != FA_OK) return s;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
 
   const int BH = B * H;
   alignas(64) CUtensorMap tq, tk, tv;
   if ((s = make_bf16_tile_map(&tq, q, d, N, BH)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&tk, k, d, N, BH)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&tv, v, d, N, BH)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tk, k, d, N, B * Hkv)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tv, v, d, N, B * Hkv)) != FA_OK) return s;
 
   fa::FwdParams p;
   p.o = o;
   p.lse = lse;
   p.BH = BH;
+  p.H = H;
+  p.Hkv = Hkv;
   p.N = N;
   p.n_pairs = (N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -308,20 +353,37 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return fa::bwd_workspace_bytes(B * H, N, d);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int N, int d,
-                 float scale, int causal, void* stream) {
+size_t fa_bwd_gqa_workspace_size(int B, int H, int Hkv, int N, int d) {
+  if (check_sizes(B, H, N, d, 1.f, 0) != FA_OK || Hkv < 1 || H % Hkv != 0) return 0;
+  return fa::bwd_gqa_workspace_bytes(B, H, Hkv, N, d);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, fa_dtype o_dtype, void* stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, o_dtype, stream);
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N,
+                     int d, float scale, int causal, void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
   fa_status s = check_sizes(B, H, N, d, scale, causal);
   if (s != FA_OK) return s;
-  if (ws_bytes < fa::bwd_workspace_bytes(B * H, N, d)) return FA_ERR_INVALID_ARG;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (ws_bytes < fa::bwd_gqa_workspace_bytes(B, H, Hkv, N, d)) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B * H, N, scale, causal, st);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, st);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  return fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, H, N, d, scale, causal, stream);
 }
 
 int fa_last_cuda_error(void) { return t_last_cuda_error; }
@@ -366,8 +428,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B * H, N, scale, causal, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B * H, N, scale, causal, st);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, causal, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, causal, st);
 }
 
 }  // extern "C"

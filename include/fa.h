@@ -129,6 +129,36 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          float scale, int causal, void* stream);
 
 /*
+ * Grouped-query / multi-query attention (several query heads share one K/V
+ * head; "FlashAttention原理：从原始Attention到FlashAttention", blog.csdn.net,
+ * related-article notes on MQA/GQA). q, o, dO, dq are [B, H, N, d]; k, v,
+ * dk, dv are [B, Hkv, N, d] with H % Hkv == 0, and query head h reads K/V
+ * head h / (H / Hkv). Hkv == H is ordinary multi-head attention (what fa_fwd
+ * and fa_bwd compute); Hkv == 1 is multi-query attention. dk and dv hold the
+ * gradient of each shared K/V head, summed over its group, accumulated on
+ * chip over the query heads one CTA covers. lse is [B, H, N]. Every other
+ * convention is fa_fwd's and fa_bwd's; Hkv < 1 or H % Hkv != 0 gives
+ * FA_ERR_INVALID_ARG.
+ *
+ * When few K/V heads would leave the GPU short of CTAs, fa_bwd_gqa splits
+ * each group's query heads over several CTAs, which add their partial dK and
+ * dV into fp32 accumulators in the workspace (zeroed by the row-dot kernel)
+ * and two more launches of the convert kernel write dk and dv. Its workspace
+ * is fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) bytes: fa_bwd_workspace_size
+ * (B, H, N, d) plus, when Hkv < H, two fp32 [B, Hkv, N, d] arrays, each
+ * rounded up to 256 bytes (0 for invalid sizes). The split adds fp32 sums in
+ * a run-dependent order, so dk and dv may then differ between runs in the
+ * last bits.
+ */
+size_t fa_bwd_gqa_workspace_size(int B, int H, int Hkv, int N, int d);
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Hkv, int N, int d, float scale, int causal, fa_dtype o_dtype,
+                     void* stream);
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                     int B, int H, int Hkv, int N, int d, float scale, int causal, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.

@@ -14,6 +14,7 @@ FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
 def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
+                          "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_gqa_workspace_size",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
                           "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
@@ -124,3 +125,28 @@ def test_noalloc_scratch_size_matches_header():
     with open(fa.HEADER_PATH) as f:
         m = re.search(r"#define FA_NOALLOC_SCRATCH_BYTES \((\d+)u \* 1024u \* 1024u\)", f.read())
     assert m and int(m.group(1)) * 1024 * 1024 == fa.FA_NOALLOC_SCRATCH_BYTES
+
+
+@pytest.mark.parametrize("H,Hkv", [(8, 3), (4, 0), (4, -2), (2, 4)])
+def test_gqa_rejects_bad_head_counts(H, Hkv):
+    assert fa.fa_fwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, Hkv, 16, 64, 0.1, 0, fa.FA_BF16,
+                         None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 1, H, Hkv, 16, 64,
+                         0.1, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_gqa_workspace_size_formula():
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for B, H, Hkv, N, d in ((1, 16, 16, 1000, 128), (2, 8, 2, 777, 64), (1, 16, 1, 16384, 128)):
+        base = fa.fa_bwd_workspace_size(B, H, N, d)
+        extra = 0 if Hkv == H else 2 * up(B * Hkv * N * d * 4)
+        assert fa.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) == base + extra
+    assert fa.fa_bwd_gqa_workspace_size(1, 8, 3, 64, 64) == 0
+    assert fa.fa_bwd_gqa_workspace_size(1, 8, 0, 64, 64) == 0
+
+
+def test_gqa_bwd_rejects_small_workspace():
+    need = fa.fa_bwd_gqa_workspace_size(1, 8, 2, 256, 64)
+    assert need > fa.fa_bwd_workspace_size(1, 8, 256, 64)
+    assert fa.fa_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 1, 8, 2, 256, 64,
+                         0.1, 0, None) == fa.FA_ERR_INVALID_ARG

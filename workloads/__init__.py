@@ -74,19 +74,22 @@ WORKLOADS: Dict[str, Workload] = {
 
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0,
-                with_grad_out: bool = True):
+                with_grad_out: bool = True, kv_heads: Optional[int] = None):
     """Draw Q, K, V (and dO) as bf16 CPU tensors of shape [B, H, N, d].
 
-    Returns a dict with keys ``q``, ``k``, ``v`` and, if requested, ``do``.
+    With ``kv_heads`` set (grouped-query attention), K and V are
+    [B, kv_heads, N, d] instead. Returns a dict with keys ``q``, ``k``, ``v``
+    and, if requested, ``do``.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(int(seed))
     shape = (B, H, N, d)
+    kv_shape = shape if kv_heads is None else (B, int(kv_heads), N, d)
     out = {}
     for name in ("q", "k", "v", "do"):
         if name == "do" and not with_grad_out:
             break
-        t = torch.randn(shape, generator=g, dtype=torch.float32)
+        t = torch.randn(kv_shape if name in ("k", "v") else shape, generator=g, dtype=torch.float32)
         if name in ("q", "k") and qk_std != 1.0:
             t.mul_(qk_std)
         out[name] = t.to(torch.bfloat16)
