@@ -22,6 +22,11 @@ Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
   (MQA/GQA): the definition with K/V heads repeated per group; dK, dV summed
   over the group. Pinned by: central finite differences with respect to the
   shared K/V tensors, the MQA closed form for Q = 0, and group size 1 = MHA.
+- ``window=(wl, wr)`` on the forward and backward functions: the local-window
+  (band) mask i - wl <= j <= i + wr. Pinned by: a pure-Python per-row
+  computation over the explicitly listed visible keys, the closed form for
+  wl = wr = 0 (O = V, lse = scale q.k), unbounded windows equal to the full and
+  causal masks, and central finite differences of the backward.
 - ``blockwise_online_softmax_attention`` the tiled merge with running max and
   running sum. Pinned by: equality with the full-row softmax on tiny inputs,
   for several block sizes.
@@ -36,6 +41,7 @@ from .attention import (  # noqa: F401
     attention_backward_rows,
     attention_backward_gqa,
     attention_forward_gqa,
+    band_visible,
     causal_visible,
 )
 from .online_softmax import blockwise_online_softmax_attention  # noqa: F401

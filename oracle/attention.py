@@ -19,6 +19,12 @@ Readings of points the pages leave open:
 - causal mask: key j is visible to query i iff j <= i (square problem, N_q =
   N_k). Masked logits are -inf before the row max, so they contribute exactly
   0. With j <= i no row is ever fully masked.
+- local window ("Local-Window" among the sparse extensions listed in
+  "FlashAttention：优化大模型训练的内存与计算效率", cnnetsun.cn, section 6.1;
+  the page gives only the name): ``window = (wl, wr)`` makes key j visible to
+  query i iff i - wl <= j <= i + wr, a negative bound meaning no limit on that
+  side. It combines with ``causal`` by intersection; (-1, 0) is the causal
+  mask. With wl, wr >= 0 the diagonal is always visible, so no row is empty.
 - lse is the natural logarithm of sum_j exp(scale * q_i . k_j) over visible j:
   lse_i = m_i + ln(l_i) where m_i is the row max of the scaled logits and l_i
   the row sum of exp(S - m_i). The pages say only that the forward stores the
@@ -58,12 +64,27 @@ def causal_visible(rows: np.ndarray, n_keys: int) -> np.ndarray:
     return np.arange(n_keys)[None, :] <= np.asarray(rows)[:, None]
 
 
+def band_visible(rows: np.ndarray, n_keys: int, wl: int, wr: int) -> np.ndarray:
+    """Boolean [len(rows), n_keys] matrix: key j visible to query i iff
+    i - wl <= j <= i + wr (a negative wl or wr: no bound on that side)."""
+    j = np.arange(n_keys)[None, :]
+    i = np.asarray(rows)[:, None]
+    vis = np.ones((len(rows), n_keys), dtype=bool)
+    if wl >= 0:
+        vis &= j >= i - wl
+    if wr >= 0:
+        vis &= j <= i + wr
+    return vis
+
+
 def _scores(q_rows: np.ndarray, k: np.ndarray, scale: float, rows: np.ndarray,
-            causal: bool) -> np.ndarray:
+            causal: bool, window=None) -> np.ndarray:
     """S = scale * Q K^T for the given query rows, masked entries set to -inf."""
     s = (q_rows @ k.T) * scale
     if causal:
         s = np.where(causal_visible(rows, k.shape[0]), s, -np.inf)
+    if window is not None:
+        s = np.where(band_visible(rows, k.shape[0], window[0], window[1]), s, -np.inf)
     return s
 
 
@@ -75,22 +96,23 @@ def _softmax_rows(s: np.ndarray):
     return e / l, m[:, 0], l[:, 0]
 
 
-def _forward_head(q, k, v, scale, causal, rows):
+def _forward_head(q, k, v, scale, causal, rows, window=None):
     o = np.empty((len(rows), v.shape[1]))
     lse = np.empty(len(rows))
     for c0 in range(0, len(rows), _CHUNK):
         r = rows[c0:c0 + _CHUNK]
-        s = _scores(q[r], k, scale, r, causal)
+        s = _scores(q[r], k, scale, r, causal, window)
         p, m, l = _softmax_rows(s)
         o[c0:c0 + len(r)] = p @ v
         lse[c0:c0 + len(r)] = m + np.log(l)
     return o, lse
 
 
-def attention_forward(q, k, v, scale: float, causal: bool):
+def attention_forward(q, k, v, scale: float, causal: bool, window=None):
     """O and lse of exact attention.
 
-    q, k, v: [B, H, N, d]. Returns (O [B, H, N, d] fp64, lse [B, H, N] fp64).
+    q, k, v: [B, H, N, d]; window: None or (wl, wr), see the module notes.
+    Returns (O [B, H, N, d] fp64, lse [B, H, N] fp64).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, _ = q.shape
@@ -99,11 +121,11 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     rows = np.arange(N)
     for b in range(B):
         for h in range(H):
-            o[b, h], lse[b, h] = _forward_head(q[b, h], k[b, h], v[b, h], scale, causal, rows)
+            o[b, h], lse[b, h] = _forward_head(q[b, h], k[b, h], v[b, h], scale, causal, rows, window)
     return o, lse
 
 
-def attention_forward_rows(q, k, v, scale: float, causal: bool, heads, rows):
+def attention_forward_rows(q, k, v, scale: float, causal: bool, heads, rows, window=None):
     """O and lse for selected (b, h) heads and query rows only.
 
     heads: list of (b, h) pairs; rows: 1-D array of query indices.
@@ -113,13 +135,13 @@ def attention_forward_rows(q, k, v, scale: float, causal: bool, heads, rows):
     outs_o, outs_l = [], []
     for (b, h) in heads:
         qh, kh, vh = _f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h])
-        o, l = _forward_head(qh, kh, vh, scale, causal, rows)
+        o, l = _forward_head(qh, kh, vh, scale, causal, rows, window)
         outs_o.append(o)
         outs_l.append(l)
     return np.stack(outs_o), np.stack(outs_l)
 
 
-def _backward_head(q, k, v, do, scale, causal, rows=None):
+def _backward_head(q, k, v, do, scale, causal, rows=None, window=None):
     """Gradients from the query rows ``rows`` (all rows if None) of one head.
 
     dQ is returned for those rows only; dK and dV are the contributions of
@@ -131,7 +153,7 @@ def _backward_head(q, k, v, do, scale, causal, rows=None):
     dv = np.zeros_like(v)
     for c0 in range(0, len(rows), _CHUNK):
         r = rows[c0:c0 + _CHUNK]
-        s = _scores(q[r], k, scale, r, causal)
+        s = _scores(q[r], k, scale, r, causal, window)
         p, _, _ = _softmax_rows(s)          # recomputed from the definition
         dv += p.T @ do[r]                   # dV = P^T dO
         dp = do[r] @ v.T                    # dP = dO V^T
@@ -153,15 +175,17 @@ def attention_backward_rows(q, k, v, do, scale: float, causal: bool, heads, rows
     return tuple(np.stack([r[i] for r in res]) for i in range(3))
 
 
-def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
+def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, window=None):
     """dQ, dK, dV of exact attention for upstream gradient dO.
 
     All inputs [B, H, N, d]. If ``heads`` (a list of (b, h)) is given, only those
     heads are computed and the results are stacked as [len(heads), N, d].
+    window: None or (wl, wr), see the module notes.
     """
     if heads is not None:
         res = [
-            _backward_head(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(do[b, h]), scale, causal)
+            _backward_head(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(do[b, h]), scale, causal,
+                           window=window)
             for (b, h) in heads
         ]
         return tuple(np.stack([r[i] for r in res]) for i in range(3))
@@ -170,7 +194,8 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
     dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
     for b in range(B):
         for h in range(H):
-            dq[b, h], dk[b, h], dv[b, h] = _backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal)
+            dq[b, h], dk[b, h], dv[b, h] = _backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal,
+                                                          window=window)
     return dq, dk, dv
 
 
@@ -187,18 +212,18 @@ def _repeat_kv(x, group: int) -> np.ndarray:
     return np.repeat(_f64(x), group, axis=1)
 
 
-def attention_forward_gqa(q, k, v, scale: float, causal: bool):
+def attention_forward_gqa(q, k, v, scale: float, causal: bool, window=None):
     """q [B, H, N, d]; k, v [B, H_kv, N, d] with H % H_kv == 0."""
     H, Hkv = q.shape[1], k.shape[1]
     assert H % Hkv == 0
     g = H // Hkv
-    return attention_forward(q, _repeat_kv(k, g), _repeat_kv(v, g), scale, causal)
+    return attention_forward(q, _repeat_kv(k, g), _repeat_kv(v, g), scale, causal, window)
 
 
-def attention_backward_gqa(q, k, v, do, scale: float, causal: bool):
+def attention_backward_gqa(q, k, v, do, scale: float, causal: bool, window=None):
     """dQ [B, H, N, d]; dK, dV [B, H_kv, N, d] (summed over each group)."""
     B, H, N, d = q.shape
     Hkv = k.shape[1]
     g = H // Hkv
-    dq, dk, dv = attention_backward(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal)
+    dq, dk, dv = attention_backward(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal, window=window)
     return dq, dk.reshape(B, Hkv, g, N, -1).sum(axis=2), dv.reshape(B, Hkv, g, N, -1).sum(axis=2)

@@ -78,8 +78,8 @@ def test_mask_off_by_one_is_caught(monkeypatch):
 def test_transposed_p_in_forward_is_caught(monkeypatch):
     orig = att._forward_head
 
-    def bad(q, k, v, scale, causal, rows):
-        s = att._scores(q[rows], k, scale, rows, causal)
+    def bad(q, k, v, scale, causal, rows, window=None):
+        s = att._scores(q[rows], k, scale, rows, causal, window)
         p, m, l = att._softmax_rows(s)
         return p.T @ v, m + np.log(l)
 
@@ -100,10 +100,10 @@ def test_lse_missing_max_is_caught(monkeypatch):
 
 
 def _patch_backward(monkeypatch, variant):
-    def bwd(q, k, v, do, scale, causal):
+    def bwd(q, k, v, do, scale, causal, rows=None, window=None):
         N = q.shape[0]
         r = np.arange(N)
-        s = att._scores(q, k, scale, r, causal)
+        s = att._scores(q, k, scale, r, causal, window)
         p, _, _ = att._softmax_rows(s)
         dp = do @ v.T
         dd = np.sum(p * dp, axis=1, keepdims=True)
@@ -135,6 +135,37 @@ def test_backward_mistakes_are_caught(monkeypatch, variant):
 
 def test_scale_misapplied_is_caught(monkeypatch):
     orig_scores = att._scores
-    monkeypatch.setattr(att, "_scores", lambda q, k, scale, rows, causal:
-                        orig_scores(q, k, math.sqrt(scale), rows, causal))
+    monkeypatch.setattr(att, "_scores", lambda q, k, scale, rows, causal, window=None:
+                        orig_scores(q, k, math.sqrt(scale), rows, causal, window))
     assert not _golden_ok()
+
+
+def _window_ok():
+    """The band mask against an explicit per-row listing of visible keys."""
+    n, d, scale = 9, 3, 0.7
+    q, k, v = (_rand((n, d), s) for s in (11, 12, 13))
+    for wl, wr in ((2, 1), (0, 3), (3, 0)):
+        o, lse = att.attention_forward(q[None, None], k[None, None], v[None, None], scale, False, window=(wl, wr))
+        for i in range(n):
+            js = list(range(max(0, i - wl), min(n, i + wr + 1)))
+            x = scale * (k[js] @ q[i])
+            w = np.exp(x - x.max())
+            if not (np.allclose(o[0, 0, i], w @ v[js] / w.sum(), rtol=0, atol=1e-13)
+                    and abs(lse[0, 0, i] - (x.max() + np.log(w.sum()))) < 1e-13):
+                return False
+    return True
+
+
+def test_unmutated_window_passes():
+    assert _window_ok()
+
+
+@pytest.mark.parametrize("side", ["left", "right"])
+def test_window_off_by_one_is_caught(monkeypatch, side):
+    orig = att.band_visible
+
+    def bad(rows, n, wl, wr):
+        return orig(rows, n, wl - 1 if side == "left" else wl, wr + 1 if side == "right" else wr)
+
+    monkeypatch.setattr(att, "band_visible", bad)
+    assert not _window_ok()

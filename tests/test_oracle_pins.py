@@ -337,3 +337,81 @@ def test_gqa_group_size_one_is_mha():
     np.testing.assert_array_equal(l1, l2)
     for a, b in zip(attention_backward_gqa(q, k, v, do, 0.5, True), attention_backward(q, k, v, do, 0.5, True)):
         np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------- local-window (band) mask
+
+def _per_row_window_attention(q, k, v, scale, wl, wr):
+    """Row by row in plain Python: list the visible keys explicitly (the band
+    i - wl <= j <= i + wr, clipped to the sequence), take their exponentials
+    relative to the largest logit, and average V with those weights."""
+    n, d = len(q), len(q[0])
+    o, lse = [], []
+    for i in range(n):
+        lo = 0 if wl < 0 else max(0, i - wl)
+        hi = n - 1 if wr < 0 else min(n - 1, i + wr)
+        logits = [scale * sum(q[i][c] * k[j][c] for c in range(d)) for j in range(lo, hi + 1)]
+        mx = max(logits)
+        w = [math.exp(x - mx) for x in logits]
+        tot = sum(w)
+        o.append([sum(w[t] * v[lo + t][c] for t in range(len(w))) / tot for c in range(v.shape[1])])
+        lse.append(mx + math.log(tot))
+    return np.array(o), np.array(lse)
+
+
+@pytest.mark.parametrize("wl,wr", [(0, 0), (1, 0), (2, 3), (3, -1), (-1, 2), (5, 5), (0, -1)])
+def test_window_against_per_row_python(wl, wr):
+    n, d = 9, 3
+    q, k, v = (_rand((n, d), s) for s in (81, 82, 83))
+    o, lse = attention_forward(_as4(q), _as4(k), _as4(v), 0.7, False, window=(wl, wr))
+    o_ref, lse_ref = _per_row_window_attention(q, k, v, 0.7, wl, wr)
+    assert np.allclose(o[0, 0], o_ref, rtol=0, atol=1e-13)
+    assert np.allclose(lse[0, 0], lse_ref, rtol=0, atol=1e-13)
+
+
+def test_window_zero_width_closed_form():
+    """wl = wr = 0: each query sees only its own key, so O = V and
+    lse_i = scale * q_i . k_i exactly."""
+    n, d = 12, 5
+    q, k, v = (_rand((1, 2, n, d), s) for s in (84, 85, 86))
+    o, lse = attention_forward(q, k, v, 0.3, False, window=(0, 0))
+    assert np.array_equal(o, v)
+    assert np.allclose(lse, 0.3 * np.sum(q * k, axis=-1), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_window_unbounded_equals_full_and_causal(causal):
+    n, d = 33, 8
+    q, k, v = (_rand((1, 1, n, d), s) for s in (87, 88, 89))
+    o_ref, lse_ref = attention_forward(q, k, v, 0.5, causal)
+    windows = [(-1, -1), (n, n), (n - 1, -1)] + ([(-1, 0), (n, 0)] if causal else [])
+    for w in windows:
+        wc = (w[0], 0) if causal and w[1] < 0 else w
+        o, lse = attention_forward(q, k, v, 0.5, False, window=wc) if causal and wc[1] == 0 else \
+            attention_forward(q, k, v, 0.5, causal, window=w)
+        assert np.array_equal(o, o_ref) and np.array_equal(lse, lse_ref), w
+
+
+@pytest.mark.parametrize("wl,wr", [(2, 0), (1, 2), (0, 0)])
+def test_window_backward_central_finite_differences(wl, wr):
+    n, d, scale, h = 8, 3, 0.6, 1e-6
+    q, k, v, do = (_rand((1, 1, n, d), s) for s in (91, 92, 93, 94))
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward(q_, k_, v_, scale, False, window=(wl, wr))
+        return float(np.sum(o * do))
+
+    grads = attention_backward(q, k, v, do, scale, False, window=(wl, wr))
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        if wl == 0 and wr == 0 and which in (0, 1):
+            assert np.max(np.abs(g)) == 0.0 and np.max(np.abs(num)) < 1e-9
+        else:
+            err = np.max(np.abs(num - g)) / np.max(np.abs(g))
+            assert err <= 1e-6, (which, err)
