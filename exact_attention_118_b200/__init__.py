@@ -35,6 +35,9 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_gqa_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+    "fa_bwd_window": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _F, _I, _I,
+                           _P]),
     "fa_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
@@ -96,6 +99,16 @@ def fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) -> int:
     return _lib.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
 
 
+def fa_fwd_window(q, k, v, o, lse, B, H, Hkv, N, d, scale, window_left, window_right, o_dtype, stream) -> int:
+    return _lib.fa_fwd_window(q, k, v, o, lse, B, H, Hkv, N, d, scale, window_left, window_right, o_dtype, stream)
+
+
+def fa_bwd_window(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, d, scale, window_left,
+                  window_right, stream) -> int:
+    return _lib.fa_bwd_window(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, d, scale,
+                              window_left, window_right, stream)
+
+
 def fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, o_dtype, stream) -> int:
     return _lib.fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, o_dtype, stream)
 
@@ -152,10 +165,22 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
-def attention_forward(q, k, v, scale=None, causal=False, out_fp32=False, out=None, lse=None):
+def _window(causal, window):
+    if window is None:
+        return -1, (0 if causal else -1)
+    wl, wr = (int(x) for x in window)
+    if causal:
+        wr = 0
+    return wl, wr
+
+
+def attention_forward(q, k, v, scale=None, causal=False, out_fp32=False, out=None, lse=None, window=None):
     """O, lse = attention(q, k, v) on the GPU. q: contiguous bf16 CUDA tensor
     [B, H, N, d]; k, v: [B, Hkv, N, d] with H % Hkv == 0 (Hkv = H for
-    multi-head attention). Returns (O [B,H,N,d] bf16 or fp32, lse [B,H,N] fp32)."""
+    multi-head attention). window: None or (wl, wr), key j visible to query i
+    iff i - wl <= j <= i + wr (negative: unbounded), intersected with the
+    causal mask when causal is set. Returns (O [B,H,N,d] bf16 or fp32, lse
+    [B,H,N] fp32)."""
     import torch
 
     B, H, N, d = _shape(q)
@@ -169,15 +194,17 @@ def attention_forward(q, k, v, scale=None, causal=False, out_fp32=False, out=Non
         out = torch.empty((B, H, N, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Hkv, N, d,
-                    float(scale), int(bool(causal)), FA_F32 if out.dtype == torch.float32 else FA_BF16,
-                    _stream_ptr(torch, q.device))
+    wl, wr = _window(causal, window)
+    st = fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Hkv, N, d,
+                       float(scale), wl, wr, FA_F32 if out.dtype == torch.float32 else FA_BF16,
+                       _stream_ptr(torch, q.device))
     _check(st, "fa_fwd")
     return out, lse
 
 
-def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None):
-    """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of attention on the GPU, all bf16."""
+def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=None, window=None):
+    """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of attention on the GPU, all bf16
+    (masks as in attention_forward)."""
     import torch
 
     B, H, N, d = _shape(q)
@@ -196,9 +223,10 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=
     ws_bytes = fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    st = fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                    B, H, Hkv, N, d, float(scale), int(bool(causal)), _stream_ptr(torch, q.device))
+    wl, wr = _window(causal, window)
+    st = fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                       B, H, Hkv, N, d, float(scale), wl, wr, _stream_ptr(torch, q.device))
     _check(st, "fa_bwd")
     return dq, dk, dv
 

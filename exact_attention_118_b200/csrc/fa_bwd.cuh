@@ -136,6 +136,7 @@ struct BwdParams {
   int H;          // query heads
   int Hkv;        // K/V heads; query heads [g*H/Hkv, (g+1)*H/Hkv) share K/V head g
   int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv)
+  int wl, wr;     // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
   int N;
   int n_kv;          // ceil(N / 128)
   int n_q;           // ceil(N / 64)
@@ -179,7 +180,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   // Causal: key tile 0 sees every query tile, so low j first (heaviest).
   int j, unit;
-  if (CAUSAL) {
+  if (MASK == kMaskCausal) {
     j = static_cast<int>(blockIdx.x) / p.BH;
     unit = static_cast<int>(blockIdx.x) % p.BH;
   } else {
@@ -232,8 +233,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int bkv = unit / p.n_split;
   const int group = p.H / p.Hkv / p.n_split;  // query heads of this CTA
   const int qh0 = (bkv / p.Hkv) * p.H + (bkv % p.Hkv) * (p.H / p.Hkv) + (unit % p.n_split) * group;
-  const int i_start = CAUSAL ? 2 * j : 0;  // first 64-query tile with a visible query
-  const int n_iq = p.n_q - i_start;        // query tiles per head (>= 1 since 128*j < N)
+  // 64-query tiles [i_start, i_end) that see a key of this tile; never empty,
+  // since key 128*j < N sees itself.
+  int i_start = 0, i_end = p.n_q;
+  if (MASK == kMaskCausal) i_start = 2 * j;
+  if (MASK == kMaskBand) {
+    i_start = max(0, j * 128 - p.wr) / 64;
+    i_end = min(p.n_q, min(j * 128 + 127 + p.wl, N - 1) / 64 + 1);
+  }
+  const int n_iq = i_end - i_start;  // query tiles per head
   const int n_it = group * n_iq;
   auto q_start = [&](int it) { return (i_start + it % n_iq) * 64; };
   auto q_head = [&](int it) { return qh0 + it / n_iq; };
@@ -423,7 +431,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const float4* lse2 = reinterpret_cast<const float4*>(smem + L::kStat + s * 512);
       const float4* dd = lse2 + 16;
-      const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (CAUSAL && j * 128 + 127 > q0);
+      const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (MASK == kMaskCausal && j * 128 + 127 > q0) ||
+                        (MASK == kMaskBand && (j * 128 + 127 > q0 + p.wr || j * 128 < q0 + 63 - p.wl));
       float pr[64];
       {
         uint32_t sv[64];
@@ -443,7 +452,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int qi = q0 + c;
-          const bool vis = (qi < N) && (kj < N) && (!CAUSAL || kj <= qi);
+          const bool vis = (qi < N) && (kj < N) && (MASK != kMaskCausal || kj <= qi) &&
+                           (MASK != kMaskBand || (kj >= qi - p.wl && kj <= qi + p.wr));
           if (!vis) pr[c] = 0.f;
         }
       }

@@ -8,7 +8,9 @@
 // end (the second FlashAttention's cut of non-matmul work, blog section 二.7);
 // query tiles form the outer loop and key/value tiles the inner loop (same
 // section); tiles wholly above the causal diagonal are never visited (same
-// section, third point). Only O and lse reach global memory.
+// section, third point). Only O and lse reach global memory. A local window
+// (the band i - wl <= j <= i + wr, "Local-Window" in cnnetsun.cn section 6.1)
+// visits only the K/V tiles the band touches, each query tile its own range.
 //
 // One CTA owns two 128-row query tiles of one (batch, head) and streams the
 // K/V tiles of that head through a shared-memory ring:
@@ -43,6 +45,7 @@ struct FwdParams {
   int N;
   int n_pairs;       // ceil(N / 256): CTAs per (batch, head)
   float scale_log2;  // scale * log2(e)
+  int wl, wr;        // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
 };
 
 template <int D>
@@ -62,7 +65,7 @@ struct FwdLayout {
 constexpr int kFwdThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D, bool CAUSAL, bool OF32>
+template <int D, int MASK, bool OF32>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // Causal: heaviest query tiles first across all heads. Otherwise head-major
   // so CTAs that read the same K/V run together and share it through L2.
   int pair, bh;
-  if (CAUSAL) {
+  if (MASK == kMaskCausal) {
     pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / p.BH;
     bh = static_cast<int>(blockIdx.x) % p.BH;
   } else {
@@ -102,13 +105,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
   const int q0 = pair * 256;
   const int n_kv = (N + 127) / 128;
-  int n_t[2];
+  // K/V tiles [lo, hi) that query tile t needs. The CTA streams tiles j0 + j,
+  // j in [0, J); tile t takes part in steps [a_t, b_t) of that stream. The
+  // two ranges overlap or touch (the diagonal tile of query tile 0 reaches
+  // the first tile query tile 1 needs), so the stream has no gaps.
+  int a_t[2], b_t[2], j0 = 0;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qs = q0 + 128 * t;
-    n_t[t] = (qs >= N) ? 0 : (CAUSAL ? min(n_kv, qs / 128 + 1) : n_kv);
+    int lo = 0, hi = 0;
+    if (qs < N) {
+      hi = n_kv;
+      if (MASK == kMaskCausal) hi = min(n_kv, qs / 128 + 1);
+      if (MASK == kMaskBand) {
+        lo = max(0, qs - p.wl) / 128;
+        hi = min(n_kv, (min(qs + 127, N - 1) + p.wr) / 128 + 1);
+      }
+    }
+    if (t == 0) j0 = lo;
+    a_t[t] = (hi > lo) ? lo - j0 : 0;
+    b_t[t] = (hi > lo) ? hi - j0 : 0;
   }
-  const int J = max(n_t[0], n_t[1]);
+  const int J = max(b_t[0], b_t[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -151,12 +169,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(k_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, j * 128, bkv);
+          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, (j0 + j) * 128, bkv);
         k_issued = j + 1;
         if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, j * 128, bkv);
+          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, (j0 + j) * 128, bkv);
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.
@@ -195,7 +213,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0) {
+          if (a_t[t] == 0 && b_t[t] > 0) {
             issue_s(t, 0);
             mma_commit(s_full + t);
           }
@@ -208,14 +226,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int jn = j + 1, sn = jn % S;
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
-          if (j < n_t[t]) {
-            if (!(ok = wait_parity(p_full + t, j & 1, abort_flag))) break;
+          if (j >= a_t[t] && j < b_t[t]) {
+            if (!(ok = wait_parity(p_full + t, (j - a_t[t]) & 1, abort_flag))) break;
             tc_fence_after();
-            issue_pv(t, s, j > 0);
+            issue_pv(t, s, j > a_t[t]);
             mma_commit(o_full + t);
           }
           if (t == 1) mma_commit(v_empty + s);
-          if (jn < n_t[t]) {
+          if (jn >= a_t[t] && jn < b_t[t]) {
             if (!k_next) {
               if (!(ok = wait_parity(k_full + sn, (jn / S) & 1, abort_flag))) break;
               tc_fence_after();
@@ -240,7 +258,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * D;
-    const int nt = n_t[t];
+    const int a_me = t ? a_t[1] : a_t[0];  // selects, not a local-memory index
+    const int nt = (t ? b_t[1] : b_t[0]) - a_me;
     const float lam = p.scale_log2;
 
     float m = -INFINITY;  // running max, log2 units
@@ -261,10 +280,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       }
-      const int kb = j * 128;
-      if (kb + 128 > N || (CAUSAL && kb + 127 > q0 + 128 * t)) {
+      const int kb = (j0 + a_me + j) * 128;
+      if (MASK == kMaskBand) {
+        const int qs = q0 + 128 * t;
+        if (kb + 128 > N || kb + 127 > qs + p.wr || kb < qs + 127 - p.wl) {
+          const int hi = min(N - kb, qi + p.wr - kb + 1), lo = qi - p.wl - kb;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= hi || c < lo) s[c] = -INFINITY;
+        }
+      } else if (kb + 128 > N || (MASK == kMaskCausal && kb + 127 > q0 + 128 * t)) {
         int lim = N - kb;
-        if (CAUSAL) lim = min(lim, qi - kb + 1);
+        if (MASK == kMaskCausal) lim = min(lim, qi - kb + 1);
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= lim) s[c] = -INFINITY;
@@ -285,7 +312,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_blk;
         rescale = true;
       }
-      const float neg_m = -m;
+      // A band can hide a whole tile from some rows: while a row has seen no
+      // visible key its m is -inf and its p must come out 0, not NaN.
+      const float neg_m = (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m;
       float rs0 = 0.f, rs1 = 0.f;
       uint32_t pk[64];
 #pragma unroll

@@ -115,16 +115,39 @@ unsigned helper_grid(long long threads_needed) {
   return static_cast<unsigned>(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
 }
 
-template <int D, bool CAUSAL, bool OF32>
+// The mask a call asks for, reduced to one of the kernels' three modes. A
+// window wider than the sequence on a side is no bound on that side, so a
+// band that bounds nothing is the unmasked kernel and a band bounded only on
+// the right at 0 is the causal one.
+struct Mask {
+  int mode, wl, wr;
+};
+Mask resolve_mask(int wl, int wr, int N) {
+  const int l = (wl < 0 || wl >= N - 1) ? N : wl;
+  const int r = (wr < 0 || wr >= N - 1) ? N : wr;
+  if (l == N && r == N) return {fa::kMaskNone, 0, 0};
+  if (l == N && r == 0) return {fa::kMaskCausal, 0, 0};
+  return {fa::kMaskBand, l, r};
+}
+
+template <int D, int MASK, bool OF32>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
                      cudaStream_t st) {
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OF32>;
+  auto kern = fa::fa_fwd_kernel<D, MASK, OF32>;
   const int smem = fa::FwdLayout<D>::kAlloc;
   if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
     return cuda_fail(e);
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
   kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, p);
   return launch_status();
+}
+
+template <int D, bool OF32>
+fa_status launch_fwd_mask(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const fa::FwdParams& p, int mode, cudaStream_t st) {
+  if (mode == fa::kMaskCausal) return launch_fwd<D, fa::kMaskCausal, OF32>(tq, tk, tv, p, st);
+  if (mode == fa::kMaskBand) return launch_fwd<D, fa::kMaskBand, OF32>(tq, tk, tv, p, st);
+  return launch_fwd<D, fa::kMaskNone, OF32>(tq, tk, tv, p, st);
 }
 
 // 2-D fp32 map of a [BH][Np] statistics array (Np >= N, a multiple of 4),
@@ -143,9 +166,9 @@ fa_status make_stat_map(CUtensorMap* m, const float* base, int N, int Np, int BH
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 fa_status launch_bwd_main(const CUtensorMap* maps, const fa::BwdParams& p, cudaStream_t st) {
-  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  auto kern = fa::fa_bwd_kernel<D, MASK>;
   const int smem = fa::BwdLayout<D>::kAlloc;
   if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
     return cuda_fail(e);
@@ -180,7 +203,7 @@ int bwd_split(int B, int H, int Hkv, int N) {
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv, int N, float scale,
-                     int causal, cudaStream_t st) {
+                     Mask mask, cudaStream_t st) {
   const int BH = B * H, BHkv = B * Hkv;
   const long long rows = static_cast<long long>(BH) * N;
   const int Np = fa::stat_stride(N);
@@ -229,12 +252,16 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.H = H;
   p.Hkv = Hkv;
   p.n_split = n_split;
+  p.wl = mask.wl;
+  p.wr = mask.wr;
   p.N = N;
   p.n_kv = (N + 127) / 128;
   p.n_q = (N + 63) / 64;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  s = causal ? launch_bwd_main<D, true>(maps, p, st) : launch_bwd_main<D, false>(maps, p, st);
+  s = mask.mode == fa::kMaskCausal ? launch_bwd_main<D, fa::kMaskCausal>(maps, p, st)
+      : mask.mode == fa::kMaskBand ? launch_bwd_main<D, fa::kMaskBand>(maps, p, st)
+                                   : launch_bwd_main<D, fa::kMaskNone>(maps, p, st);
   if (s != FA_OK) return s;
 
   // 3. dq = bf16(dQ accumulator).
@@ -313,12 +340,13 @@ const char* fa_strerror(fa_status s) {
   return "unknown status";
 }
 
-fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
-                     int N, int d, float scale, int causal, fa_dtype o_dtype, void* stream) {
+fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                        int N, int d, float scale, int window_left, int window_right, fa_dtype o_dtype,
+                        void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
   if (o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
-  fa_status s = check_sizes(B, H, N, d, scale, causal);
+  fa_status s = check_sizes(B, H, N, d, scale, 0);
   if (s != FA_OK) return s;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
@@ -338,14 +366,20 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
   p.N = N;
   p.n_pairs = (N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
+  const Mask m = resolve_mask(window_left, window_right, N);
+  p.wl = m.wl;
+  p.wr = m.wr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool f32 = (o_dtype == FA_F32);
-  if (d == 64) {
-    if (causal) return f32 ? launch_fwd<64, true, true>(tq, tk, tv, p, st) : launch_fwd<64, true, false>(tq, tk, tv, p, st);
-    return f32 ? launch_fwd<64, false, true>(tq, tk, tv, p, st) : launch_fwd<64, false, false>(tq, tk, tv, p, st);
-  }
-  if (causal) return f32 ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
-  return f32 ? launch_fwd<128, false, true>(tq, tk, tv, p, st) : launch_fwd<128, false, false>(tq, tk, tv, p, st);
+  if (d == 64)
+    return f32 ? launch_fwd_mask<64, true>(tq, tk, tv, p, m.mode, st) : launch_fwd_mask<64, false>(tq, tk, tv, p, m.mode, st);
+  return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, p, m.mode, st) : launch_fwd_mask<128, false>(tq, tk, tv, p, m.mode, st);
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                     int N, int d, float scale, int causal, fa_dtype o_dtype, void* stream) {
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  return fa_fwd_window(q, k, v, o, lse, B, H, Hkv, N, d, scale, -1, causal ? 0 : -1, o_dtype, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -363,21 +397,30 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, o_dtype, stream);
 }
 
-fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                     void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N,
-                     int d, float scale, int causal, void* stream) {
+fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H,
+                        int Hkv, int N, int d, float scale, int window_left, int window_right, void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
-  fa_status s = check_sizes(B, H, N, d, scale, causal);
+  fa_status s = check_sizes(B, H, N, d, scale, 0);
   if (s != FA_OK) return s;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (ws_bytes < fa::bwd_gqa_workspace_bytes(B, H, Hkv, N, d)) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, st);
+  const Mask m = resolve_mask(window_left, window_right, N);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, m, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, m, st);
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N,
+                     int d, float scale, int causal, void* stream) {
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  return fa_bwd_window(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, d, scale, -1,
+                       causal ? 0 : -1, stream);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -428,8 +471,9 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, causal, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, causal, st);
+  const Mask m = resolve_mask(-1, causal ? 0 : -1, N);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, m, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, m, st);
 }
 
 }  // extern "C"

@@ -280,6 +280,10 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // Pack two fp32 into bf16x2 (round to nearest even): `lo` in bits 0..15.
+// Attention masks the kernels are instantiated for. Band: key j is visible
+// to query i iff i - wl <= j <= i + wr (the local window), wl, wr >= 0.
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskBand = 2 };
+
 // Four consecutive fp32 adds into global memory, performed at L2 (no return).
 __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)

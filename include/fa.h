@@ -159,6 +159,28 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      int B, int H, int Hkv, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Local-window (band) attention ("Local-Window" among the sparse extensions of
+ * "FlashAttention：优化大模型训练的内存与计算效率", cnnetsun.cn, section 6.1):
+ * key j is visible to query i iff
+ *     i - window_left <= j <= i + window_right,
+ * a negative bound meaning no limit on that side. (-1, -1) is full attention,
+ * (-1, 0) causal attention, (w, 0) causal attention over the last w + 1
+ * keys. The diagonal is always visible, so no row is empty. Only the K/V
+ * tiles (forward) or query tiles (backward) that the band touches are
+ * visited, so the work is about N * min(N, wl + wr + 1) per head. Grouped
+ * K/V heads and every other convention are those of fa_fwd_gqa / fa_bwd_gqa
+ * (the backward workspace is fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
+ * bytes). fa_fwd_gqa and fa_bwd_gqa are these calls with (-1, causal ? 0 : -1).
+ */
+fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int Hkv, int N, int d, float scale,
+                        int window_left, int window_right, fa_dtype o_dtype, void* stream);
+fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                        int B, int H, int Hkv, int N, int d, float scale,
+                        int window_left, int window_right, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.

@@ -15,6 +15,7 @@ def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
                           "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_gqa_workspace_size",
+                          "fa_fwd_window", "fa_bwd_window",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
                           "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
@@ -150,3 +151,16 @@ def test_gqa_bwd_rejects_small_workspace():
     assert need > fa.fa_bwd_workspace_size(1, 8, 256, 64)
     assert fa.fa_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 1, 8, 2, 256, 64,
                          0.1, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_window_calls_reject_bad_arguments():
+    # bad head grouping, bad head dim, null pointer, small workspace
+    assert fa.fa_fwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 3, 64, 64, 0.1, 4, 0, fa.FA_BF16,
+                            None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, 64, 96, 0.1, 4, 0, fa.FA_BF16,
+                            None) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_window(None, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, 64, 64, 0.1, 4, 0, fa.FA_BF16,
+                            None) == fa.FA_ERR_INVALID_ARG
+    need = fa.fa_bwd_gqa_workspace_size(1, 8, 2, 256, 64)
+    assert fa.fa_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 1, 8, 2, 256, 64,
+                            0.1, 16, 16, None) == fa.FA_ERR_INVALID_ARG
