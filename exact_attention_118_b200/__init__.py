@@ -35,6 +35,10 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_gqa_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+    "fa_bwd_varlen_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _I, _F,
+                           _I, _I, _P]),
     "fa_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "fa_bwd_window": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _F, _I, _I,
                            _P]),
@@ -97,6 +101,22 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, sca
 
 def fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) -> int:
     return _lib.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, max_seqlen, T, H, Hkv, d, scale, window_left, window_right,
+                  o_dtype, stream) -> int:
+    return _lib.fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, max_seqlen, T, H, Hkv, d, scale, window_left,
+                              window_right, o_dtype, stream)
+
+
+def fa_bwd_varlen_workspace_size(B, T, H, Hkv, d) -> int:
+    return _lib.fa_bwd_varlen_workspace_size(B, T, H, Hkv, d)
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens, workspace, ws_bytes, B, max_seqlen, T, H, Hkv, d,
+                  scale, window_left, window_right, stream) -> int:
+    return _lib.fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens, workspace, ws_bytes, B, max_seqlen, T,
+                              H, Hkv, d, scale, window_left, window_right, stream)
 
 
 def fa_fwd_window(q, k, v, o, lse, B, H, Hkv, N, d, scale, window_left, window_right, o_dtype, stream) -> int:
@@ -228,6 +248,63 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, workspace=
                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
                        B, H, Hkv, N, d, float(scale), wl, wr, _stream_ptr(torch, q.device))
     _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, max_seqlen, scale=None, causal=False, window=None,
+                             out_fp32=False):
+    """Packed variable-length attention. q [T, H, d], k, v [T, Hkv, d] bf16
+    CUDA tensors; cu_seqlens int32 CUDA tensor [B + 1]. Returns (O [T, H, d],
+    lse [H, T] fp32)."""
+    import torch
+
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("expected packed [T, heads, d] tensors")
+    T, H, d = (int(x) for x in q.shape)
+    Hkv = int(k.shape[1])
+    for t, heads in ((q, H), (k, Hkv), (v, Hkv)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (T, heads, d):
+            raise ValueError("q [T,H,d] and k, v [T,Hkv,d] must be contiguous bf16 CUDA tensors")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be an int32 CUDA tensor [B + 1]")
+    B = int(cu_seqlens.numel()) - 1
+    if scale is None:
+        scale = d ** -0.5
+    out = torch.empty((T, H, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    wl, wr = _window(causal, window)
+    st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       cu_seqlens.data_ptr(), B, int(max_seqlen), T, H, Hkv, d, float(scale), wl, wr,
+                       FA_F32 if out_fp32 else FA_BF16, _stream_ptr(torch, q.device))
+    _check(st, "fa_fwd_varlen")
+    return out, lse
+
+
+def attention_backward_varlen(q, k, v, o, lse, do, cu_seqlens, max_seqlen, scale=None, causal=False, window=None,
+                              workspace=None):
+    """dQ [T, H, d], dK and dV [T, Hkv, d] of packed variable-length attention."""
+    import torch
+
+    T, H, d = (int(x) for x in q.shape)
+    Hkv = int(k.shape[1])
+    for t, shape in ((q, (T, H, d)), (k, (T, Hkv, d)), (v, (T, Hkv, d)), (o, (T, H, d)), (do, (T, H, d))):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError("q, o, dO [T,H,d] and k, v [T,Hkv,d] must be contiguous bf16 CUDA tensors")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, T):
+        raise ValueError("lse must be a contiguous fp32 tensor [H, T]")
+    B = int(cu_seqlens.numel()) - 1
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_varlen_workspace_size(B, T, H, Hkv, d)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    wl, wr = _window(causal, window)
+    st = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens.data_ptr(), workspace.data_ptr(),
+                       workspace.numel(), B, int(max_seqlen), T, H, Hkv, d, float(scale), wl, wr,
+                       _stream_ptr(torch, q.device))
+    _check(st, "fa_bwd_varlen")
     return dq, dk, dv
 
 

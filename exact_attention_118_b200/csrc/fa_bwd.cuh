@@ -62,6 +62,21 @@ inline size_t bwd_gqa_workspace_bytes(int B, int H, int Hkv, int N, int d) {
   return bwd_workspace_bytes(B * H, N, d) + (Hkv < H ? 2 * bwd_kv_acc_bytes(B, Hkv, N, d) : 0);
 }
 
+// Packed variable-length batches keep the per-row statistics per head in a
+// row of varlen_stat_stride(T, B) floats, sequence b starting at the 4-aligned
+// position round_up(cu[b], 4) + 4 b (a TMA load must start on a 16-byte
+// boundary). The +4b keeps sequences apart however their starts round; the
+// positions between one sequence's end and the next start, and the tail after
+// the last, hold zeros, so a tile that reaches past its sequence reads finite
+// values.
+inline int varlen_stat_stride(int T, int B) { return (T + 4 * B + 4 + 3) & ~3; }
+__host__ __device__ __forceinline__ int varlen_stat_start(int s0, int b) { return ((s0 + 3) & ~3) + 4 * b; }
+inline size_t bwd_varlen_workspace_bytes(int B, int T, int H, int Hkv, int d) {
+  const size_t stats = static_cast<size_t>(H) * varlen_stat_stride(T, B) * sizeof(float);
+  return align256(static_cast<size_t>(T) * H * d * sizeof(float)) + 2 * align256(stats) +
+         (Hkv < H ? 2 * bwd_kv_acc_bytes(1, Hkv, T, d) : 0);
+}
+
 // ------------------------------------------------- D = rowsum(dO*O), lse2
 // For every query row: D = sum_k dO_k * O_k, lse2 = lse * log2(e) (the
 // forward's natural-log normaliser moved to base 2 for the exp2 recompute),
@@ -110,6 +125,69 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __
     reinterpret_cast<float4*>(kv_acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// The same for a packed variable-length batch ([T, H, D] tensors, lse [H, T]),
+// one sequence per blockIdx.y step: row (token i of sequence b, head h) puts
+// D and lse2 at position varlen_stat_start(s0, b) + i of head h's statistics
+// row, zeroes its dQ accumulator row, and the gap up to the next sequence's
+// start (the whole tail, after the last sequence) is zeroed. kv_n4 float4s at
+// kv_acc are zeroed by the blocks of blockIdx.y == 0.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dot_varlen_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse,
+    float* __restrict__ lse2, float* __restrict__ dsum, float* __restrict__ dq_acc, const int* __restrict__ cu,
+    int B, int T, int H, int max_len, int Sp, float* __restrict__ kv_acc, long long kv_n4) {
+  constexpr int TPR = D / 8;
+  const int tid = static_cast<int>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int part = tid % TPR;
+  const int stride = static_cast<int>(gridDim.x) * blockDim.x / TPR;
+  for (int b = blockIdx.y; b < B; b += gridDim.y) {
+    int s0, L;
+    seq_range(cu, b, T, max_len, s0, L);
+    const int P = varlen_stat_start(s0, b);
+    const int P_end = (b == B - 1) ? Sp : varlen_stat_start(s0 + L, b + 1);
+    const int rows = L * H;
+    for (int r = tid / TPR; r < rows; r += stride) {
+      const int i = r / H, h = r - i * H;
+      const size_t off = (static_cast<size_t>(s0 + i) * H + h) * D + part * 8;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
+      const uint4 g = __ldg(reinterpret_cast<const uint4*>(dO + off));
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 af = __bfloat1622float2(a2[e]);
+        const float2 gf = __bfloat1622float2(g2[e]);
+        sum = fmaf(af.x, gf.x, sum);
+        sum = fmaf(af.y, gf.y, sum);
+      }
+#pragma unroll
+      for (int w = TPR / 2; w >= 1; w >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, w);
+      if (part == 0) {
+        const size_t so = static_cast<size_t>(h) * Sp + P + i;
+        dsum[so] = sum;
+        lse2[so] = __ldg(lse + static_cast<size_t>(h) * T + s0 + i) * 1.4426950408889634f;
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // Zero the statistics between this sequence's end and the next start.
+    const int gap = max(P_end - (P + L), 0);
+    for (int r = tid; r < gap * H; r += static_cast<int>(gridDim.x) * blockDim.x) {
+      const int h = r / gap;
+      const size_t so = static_cast<size_t>(h) * Sp + P + L + (r - h * gap);
+      dsum[so] = 0.f;
+      lse2[so] = 0.f;
+    }
+  }
+  if (blockIdx.y == 0) {
+    const long long all = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = tid; i < kv_n4; i += all)
+      reinterpret_cast<float4*>(kv_acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 // --------------------------------------------------------- dQ fp32 -> bf16
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc,
                                                                 __nv_bfloat16* __restrict__ dq, long long n8) {
@@ -137,9 +215,10 @@ struct BwdParams {
   int Hkv;        // K/V heads; query heads [g*H/Hkv, (g+1)*H/Hkv) share K/V head g
   int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv)
   int wl, wr;     // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
+  const int* cu_seqlens;  // packed variable length ([T, heads, D] tensors): [B + 1] prefix sums; else nullptr
+  int T;                  // packed rows (variable length only); N is then the longest length
   int N;
   int n_kv;          // ceil(N / 128)
-  int n_q;           // ceil(N / 64)
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
 };
@@ -215,7 +294,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int N = p.N;
 
   // Causal: key tile 0 sees every query tile, so low j first (heaviest).
   int j, unit;
@@ -230,16 +308,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // K/V head bkv (the one head, for multi-head attention): dK and dV
   // accumulate on chip over that share, and across the n_split shares in
   // fp32 global memory.
-  const int bkv = unit / p.n_split;
-  const int group = p.H / p.Hkv / p.n_split;  // query heads of this CTA
-  const int qh0 = (bkv / p.Hkv) * p.H + (bkv % p.Hkv) * (p.H / p.Hkv) + (unit % p.n_split) * group;
+  const int bkv = unit / p.n_split;  // batch * Hkv + K/V head
+  // This CTA's sequence: length N, first row s0 in the maps' row dimension.
+  // Fixed-length maps index batch*head, packed ones the head alone.
+  const bool packed = p.cu_seqlens != nullptr;
+  int N = p.N, s0 = 0;
+  if (packed) seq_range(p.cu_seqlens, bkv / p.Hkv, p.T, p.N, s0, N);
+  if (j * 128 >= N) return;  // past the end of a shorter sequence: the whole CTA leaves
+  const int kvh = packed ? bkv % p.Hkv : bkv;  // K/V head coordinate of the maps
+  // First position of this sequence in the per-row statistics (4-aligned).
+  const int stat0 = packed ? varlen_stat_start(s0, bkv / p.Hkv) : 0;
+  const int group = p.H / p.Hkv / p.n_split;   // query heads of this CTA
+  const int qh0 = (packed ? 0 : (bkv / p.Hkv) * p.H) + (bkv % p.Hkv) * (p.H / p.Hkv) + (unit % p.n_split) * group;
+  const int n_q = (N + 63) / 64;
   // 64-query tiles [i_start, i_end) that see a key of this tile; never empty,
   // since key 128*j < N sees itself.
-  int i_start = 0, i_end = p.n_q;
+  int i_start = 0, i_end = n_q;
   if (MASK == kMaskCausal) i_start = 2 * j;
   if (MASK == kMaskBand) {
     i_start = max(0, j * 128 - p.wr) / 64;
-    i_end = min(p.n_q, min(j * 128 + 127 + p.wl, N - 1) / 64 + 1);
+    i_end = min(n_q, min(j * 128 + 127 + p.wl, N - 1) / 64 + 1);
   }
   const int n_iq = i_end - i_start;  // query tiles per head
   const int n_it = group * n_iq;
@@ -290,8 +378,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_dsum);
       mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
       for (int c = 0; c < KCH; ++c) {
-        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, j * 128, bkv);
-        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, j * 128, bkv);
+        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, s0 + j * 128, kvh);
+        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, s0 + j * 128, kvh);
       }
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
@@ -301,11 +389,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint8_t* st = smem + L::kStat + s * 512;
         mbar_arrive_expect_tx(qd_full + s, kStageTx);
         for (int c = 0; c < KCH; ++c) {
-          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, q0, bhq);
-          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, q0, bhq);
+          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, s0 + q0, bhq);
+          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, s0 + q0, bhq);
         }
-        tma_load_2d(st, &tm_lse2, qd_full + s, q0, bhq);
-        tma_load_2d(st + 256, &tm_dsum, qd_full + s, q0, bhq);
+        tma_load_2d(st, &tm_lse2, qd_full + s, stat0 + q0, bhq);
+        tma_load_2d(st + 256, &tm_dsum, qd_full + s, stat0 + q0, bhq);
         issued = it + 1;
       }
       wait_parity_drain(kv_full, 0);
@@ -512,7 +600,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (ok) {
         tc_fence_after();
         const bool valid = kj < N;
-        const size_t row = static_cast<size_t>(bkv) * N + (valid ? kj : 0);
+        const int kv = valid ? kj : 0;
+        // dK/dV row of key kj, in units of D elements.
+        const size_t row = packed ? static_cast<size_t>(s0 + kv) * p.Hkv + kvh : static_cast<size_t>(bkv) * N + kv;
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e ? p.dk : p.dv) + row * D;
         float* acc = (e ? p.dk_acc : p.dv_acc) + row * D;
         const uint32_t col = e ? t_dk : t_dv;
@@ -581,7 +671,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (leader && ok) {
-          tma_reduce_add_3d(&tm_dq, stg, 0, q0 + 32 * h, bhq);
+          tma_reduce_add_3d(&tm_dq, stg, 0, s0 + q0 + 32 * h, bhq);
           bulk_commit_group();
         }
       }

@@ -12,6 +12,12 @@
 // (the band i - wl <= j <= i + wr, "Local-Window" in cnnetsun.cn section 6.1)
 // visits only the K/V tiles the band touches, each query tile its own range.
 //
+// Layouts. Fixed length: Q, O [B, H, N, D], K, V [B, Hkv, N, D]; the tensor
+// maps index (column, row, batch*head). Packed variable length: Q, O
+// [T, H, D], K, V [T, Hkv, D] with sequence b in rows [cu[b], cu[b+1]); the
+// maps index (column, packed row, head), and a CTA adds its sequence's first
+// row to every row coordinate. lse is [B, H, N] or [H, T].
+//
 // One CTA owns two 128-row query tiles of one (batch, head) and streams the
 // K/V tiles of that head through a shared-memory ring:
 //   warp 0      TMA producer: Q0, Q1 once; K_j, V_j into a KV_STAGES ring.
@@ -46,6 +52,8 @@ struct FwdParams {
   int n_pairs;       // ceil(N / 256): CTAs per (batch, head)
   float scale_log2;  // scale * log2(e)
   int wl, wr;        // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
+  const int* cu_seqlens;  // packed variable length: [B + 1] prefix sums of the lengths; else nullptr
+  int T;                  // packed rows (variable length only); N is then the longest length
 };
 
 template <int D>
@@ -91,7 +99,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int N = p.N;
 
   // Causal: heaviest query tiles first across all heads. Otherwise head-major
   // so CTAs that read the same K/V run together and share it through L2.
@@ -103,7 +110,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bh = static_cast<int>(blockIdx.x) / p.n_pairs;
     pair = static_cast<int>(blockIdx.x) % p.n_pairs;
   }
+  // This CTA's sequence: its length N and first row s0 in the maps' row
+  // dimension, and the Q/O head coordinate hq of the maps.
+  const bool packed = p.cu_seqlens != nullptr;
+  int N = p.N, s0 = 0;
+  const int hq = packed ? bh % p.H : bh;
+  if (packed) seq_range(p.cu_seqlens, bh / p.H, p.T, p.N, s0, N);
   const int q0 = pair * 256;
+  if (q0 >= N) return;  // past the end of a shorter sequence: the whole CTA leaves
   const int n_kv = (N + 127) / 128;
   // K/V tiles [lo, hi) that query tile t needs. The CTA streams tiles j0 + j,
   // j in [0, J); tile t takes part in steps [a_t, b_t) of that stream. The
@@ -155,26 +169,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       // K/V head of this query head (grouped-query attention; equal for MHA).
-      const int bkv = (bh / p.H) * p.Hkv + (bh % p.H) / (p.H / p.Hkv);
+      const int bkv = (packed ? 0 : (bh / p.H) * p.Hkv) + (bh % p.H) / (p.H / p.Hkv);
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(q_full, 2 * L::kTile);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * 64, q0 + 128 * t, bh);
+          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * 64, s0 + q0 + 128 * t, hq);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < J; ++j) {
         const int s = j % S, u = j / S;
         if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(k_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, s0 + (j0 + j) * 128, bkv);
         k_issued = j + 1;
         if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, s0 + (j0 + j) * 128, bkv);
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.
@@ -358,8 +372,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool valid = qi < N;
-        const size_t row = static_cast<size_t>(bh) * N + (valid ? qi : 0);
-        if (valid) p.lse[row] = (m + log2f(l)) * 0.69314718055994531f;
+        const int qv = valid ? qi : 0;
+        // O row (units of D elements) and lse index of query qi.
+        const size_t row = packed ? static_cast<size_t>(s0 + qv) * p.H + hq : static_cast<size_t>(bh) * N + qv;
+        const size_t li = packed ? static_cast<size_t>(hq) * p.T + s0 + qv : row;
+        if (valid) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t ov[32];

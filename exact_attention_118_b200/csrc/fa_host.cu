@@ -60,17 +60,30 @@ fa_status check_sizes(int B, int H, int N, int d, float scale, int causal) {
   return FA_OK;
 }
 
-// [BH][N][inner] row-major tensor viewed by TMA as dims {inner, N, BH}, with a
-// box of {box_inner, box_rows, 1}. Out-of-range rows of a head read as zero
-// and are clipped on store, so a ragged N never touches the next head.
-fa_status make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int inner, int N,
-                    int BH, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+// Where the rows of one call live. Fixed length: [B, heads, N, inner]
+// tensors, seen by TMA as dims {inner, N, B*heads}. Packed variable length:
+// [T, heads, inner] tensors holding sequence b in rows [cu[b], cu[b+1]), seen
+// as dims {inner, T, heads} (the head stride is then the smaller one). Either
+// way a tile is (column, row, head) and out-of-range rows read as zero and are
+// clipped on store, so a ragged tile never touches the next head.
+struct Geom {
+  int B, H, Hkv, N;         // N: the sequence length (the longest, if packed)
+  int T = 0;                // packed rows
+  const int* cu = nullptr;  // packed: [B + 1] prefix sums of the lengths (device)
+  bool packed() const { return cu != nullptr; }
+  int rows() const { return packed() ? T : N; }  // row dimension of every map
+  int map_heads(int heads) const { return packed() ? heads : B * heads; }
+};
+
+fa_status make_head_map(CUtensorMap* m, const void* base, const Geom& g, int heads, CUtensorMapDataType dt,
+                        int elem_bytes, int inner, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FA_ERR_CUDA;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(N),
-                              static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem_bytes,
-                                 static_cast<cuuint64_t>(inner) * elem_bytes * N};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(inner) * elem_bytes;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(g.rows()),
+                              static_cast<cuuint64_t>(g.map_heads(heads))};
+  const cuuint64_t strides[2] = {g.packed() ? row_bytes * heads : row_bytes,
+                                 g.packed() ? row_bytes : row_bytes * g.N};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
@@ -79,8 +92,10 @@ fa_status make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, int d, int N, int BH) {
-  return make_tmap(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+// bf16 tiles of 128 rows x 64 columns (128-byte swizzle).
+fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, const Geom& g, int heads, int d) {
+  return make_head_map(m, base, g, heads, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Caller-provided events recorded around the main backward kernel
@@ -202,61 +217,80 @@ int bwd_split(int B, int H, int Hkv, int N) {
 
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv, int N, float scale,
-                     Mask mask, cudaStream_t st) {
-  const int BH = B * H, BHkv = B * Hkv;
-  const long long rows = static_cast<long long>(BH) * N;
-  const int Np = fa::stat_stride(N);
+                     void* dq, void* dk, void* dv, void* workspace, const Geom& g, float scale, Mask mask,
+                     cudaStream_t st) {
+  // Workspace rows: the row dimension Nr of the maps times their head count.
+  const int Nr = g.rows(), BHr = g.map_heads(g.H), BHkvr = g.map_heads(g.Hkv);
+  const long long rows = static_cast<long long>(BHr) * Nr;
+  // Statistics row length: N rounded up to 4, or the packed per-sequence
+  // layout of fa::varlen_stat_stride.
+  const int Np = g.packed() ? fa::varlen_stat_stride(g.T, g.B) : fa::stat_stride(Nr);
+  const size_t stat_bytes = fa::align256(static_cast<size_t>(BHr) * Np * sizeof(float));
   char* ws = static_cast<char*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(ws);
   float* lse2 = reinterpret_cast<float*>(ws + fa::align256(rows * D * sizeof(float)));
-  float* dsum = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) +
-                                         fa::align256(static_cast<size_t>(BH) * Np * sizeof(float)));
-  const int n_split = bwd_split(B, H, Hkv, N);
+  float* dsum = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + stat_bytes);
+  const int n_split = bwd_split(g.B, g.H, g.Hkv, g.N);
   float* dk_acc = nullptr;
   float* dv_acc = nullptr;
-  const long long kv_elems = static_cast<long long>(BHkv) * N * D;
+  const long long kv_elems = static_cast<long long>(BHkvr) * Nr * D;
+  const size_t kv_acc_bytes = fa::bwd_kv_acc_bytes(1, BHkvr, Nr, D);
   if (n_split > 1) {
-    dk_acc = reinterpret_cast<float*>(ws + fa::bwd_workspace_bytes(BH, N, D));
-    dv_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(dk_acc) + fa::bwd_kv_acc_bytes(B, Hkv, N, D));
+    dk_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(dsum) + stat_bytes);
+    dv_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(dk_acc) + kv_acc_bytes);
   }
 
   // 1. D = rowsum(dO * O), lse2 = lse * log2(e), dQ (and split dK/dV) accumulators = 0.
-  fa::fa_bwd_dot_kernel<D><<<helper_grid(rows * (D / 8)), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dsum, dq_acc, rows,
-      N, Np, dk_acc, n_split > 1 ? (2 * fa::bwd_kv_acc_bytes(B, Hkv, N, D)) / 16 : 0);
+  const long long kv_n4 = n_split > 1 ? static_cast<long long>(2 * kv_acc_bytes) / 16 : 0;
+  if (g.packed()) {
+    // One grid row per sequence (strided past 65535), enough blocks across
+    // for the longest sequence, the total kept to a few waves.
+    const int gy = g.B < 65535 ? g.B : 65535;
+    long long gx = (static_cast<long long>(g.N) * g.H * (D / 8) + 255) / 256;
+    const long long cap = (static_cast<long long>(helper_grid(1LL << 40)) * 2 + gy - 1) / gy;
+    gx = gx < cap ? gx : cap;
+    fa::fa_bwd_dot_varlen_kernel<D><<<dim3(static_cast<unsigned>(gx < 1 ? 1 : gx), gy), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dsum, dq_acc, g.cu,
+        g.B, g.T, g.H, g.N, Np, dk_acc, kv_n4);
+  } else {
+    fa::fa_bwd_dot_kernel<D><<<helper_grid(rows * (D / 8)), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2, dsum, dq_acc, rows,
+        Nr, Np, dk_acc, kv_n4);
+  }
   fa_status s = launch_status();
   if (s != FA_OK) return s;
 
   // 2. Main kernel. Maps: q, k, v, dO, dQ accumulator (fp32, 32-row box), lse2, D.
   alignas(64) CUtensorMap maps[7];
-  if ((s = make_tmap(&maps[0], q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+  if ((s = make_head_map(&maps[0], q, g, g.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, 64, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
-  if ((s = make_bf16_tile_map(&maps[1], k, D, N, BHkv)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&maps[2], v, D, N, BHkv)) != FA_OK) return s;
-  if ((s = make_tmap(&maps[3], dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+  if ((s = make_bf16_tile_map(&maps[1], k, g, g.Hkv, D)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&maps[2], v, g, g.Hkv, D)) != FA_OK) return s;
+  if ((s = make_head_map(&maps[3], dO, g, g.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, 64, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
     return s;
-  if ((s = make_tmap(&maps[4], dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, D, 32,
-                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+  if ((s = make_head_map(&maps[4], dq_acc, g, g.H, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, D, 32,
+                         CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return s;
-  if ((s = make_stat_map(&maps[5], lse2, N, Np, BH)) != FA_OK) return s;
-  if ((s = make_stat_map(&maps[6], dsum, N, Np, BH)) != FA_OK) return s;
+  const int stat_dim = g.packed() ? Np : Nr;
+  if ((s = make_stat_map(&maps[5], lse2, stat_dim, Np, BHr)) != FA_OK) return s;
+  if ((s = make_stat_map(&maps[6], dsum, stat_dim, Np, BHr)) != FA_OK) return s;
   fa::BwdParams p;
   p.dk = dk;
   p.dv = dv;
   p.dk_acc = dk_acc;
   p.dv_acc = dv_acc;
-  p.BH = BHkv * n_split;
-  p.H = H;
-  p.Hkv = Hkv;
+  p.BH = g.B * g.Hkv * n_split;
+  p.H = g.H;
+  p.Hkv = g.Hkv;
   p.n_split = n_split;
   p.wl = mask.wl;
   p.wr = mask.wr;
-  p.N = N;
-  p.n_kv = (N + 127) / 128;
-  p.n_q = (N + 63) / 64;
+  p.cu_seqlens = g.cu;
+  p.T = g.T;
+  p.N = g.N;
+  p.n_kv = (g.N + 127) / 128;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   s = mask.mode == fa::kMaskCausal ? launch_bwd_main<D, fa::kMaskCausal>(maps, p, st)
@@ -323,6 +357,61 @@ fa_status noalloc_scratch(void** out) {
   return FA_OK;
 }
 
+// The forward for either layout; arguments already checked.
+fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, void* o, float* lse, int d,
+                   float scale, int window_left, int window_right, fa_dtype o_dtype, void* stream) {
+  fa_status s;
+  alignas(64) CUtensorMap tq, tk, tv;
+  if ((s = make_bf16_tile_map(&tq, q, g, g.H, d)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tk, k, g, g.Hkv, d)) != FA_OK) return s;
+  if ((s = make_bf16_tile_map(&tv, v, g, g.Hkv, d)) != FA_OK) return s;
+
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.BH = g.B * g.H;
+  p.H = g.H;
+  p.Hkv = g.Hkv;
+  p.N = g.N;
+  p.n_pairs = (g.N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const Mask m = resolve_mask(window_left, window_right, g.N);
+  p.wl = m.wl;
+  p.wr = m.wr;
+  p.cu_seqlens = g.cu;
+  p.T = g.T;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool f32 = (o_dtype == FA_F32);
+  if (d == 64)
+    return f32 ? launch_fwd_mask<64, true>(tq, tk, tv, p, m.mode, st)
+               : launch_fwd_mask<64, false>(tq, tk, tv, p, m.mode, st);
+  return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, p, m.mode, st)
+             : launch_fwd_mask<128, false>(tq, tk, tv, p, m.mode, st);
+}
+
+// The backward for either layout; arguments already checked.
+fa_status bwd_impl(const Geom& g, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, void* workspace, int d, float scale,
+                   int window_left, int window_right, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Mask m = resolve_mask(window_left, window_right, g.N);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, g, scale, m, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, g, scale, m, st);
+}
+
+// Checks shared by the variable-length calls: the prefix-sum array, the head
+// grouping and the sizes (T packed rows of H heads within int range).
+fa_status check_varlen(const int* cu_seqlens, int B, int max_seqlen, int T, int H, int Hkv, int d, float scale) {
+  if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (max_seqlen < 1) return FA_ERR_INVALID_ARG;
+  fa_status s = check_sizes(1, H, T, d, scale, 0);
+  if (s != FA_OK) return s;
+  if (B < 1 || Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+  if ((static_cast<long long>(T) + 4LL * B + 8) * H >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -350,30 +439,22 @@ fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, fl
   if (s != FA_OK) return s;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
+  return fwd_impl(Geom{B, H, Hkv, N}, q, k, v, o, lse, d, scale, window_left, window_right, o_dtype, stream);
+}
 
-  const int BH = B * H;
-  alignas(64) CUtensorMap tq, tk, tv;
-  if ((s = make_bf16_tile_map(&tq, q, d, N, BH)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&tk, k, d, N, B * Hkv)) != FA_OK) return s;
-  if ((s = make_bf16_tile_map(&tv, v, d, N, B * Hkv)) != FA_OK) return s;
-
-  fa::FwdParams p;
-  p.o = o;
-  p.lse = lse;
-  p.BH = BH;
-  p.H = H;
-  p.Hkv = Hkv;
-  p.N = N;
-  p.n_pairs = (N + 255) / 256;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  const Mask m = resolve_mask(window_left, window_right, N);
-  p.wl = m.wl;
-  p.wr = m.wr;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool f32 = (o_dtype == FA_F32);
-  if (d == 64)
-    return f32 ? launch_fwd_mask<64, true>(tq, tk, tv, p, m.mode, st) : launch_fwd_mask<64, false>(tq, tk, tv, p, m.mode, st);
-  return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, p, m.mode, st) : launch_fwd_mask<128, false>(tq, tk, tv, p, m.mode, st);
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int B, int max_seqlen, int T, int H, int Hkv, int d, float scale, int window_left,
+                        int window_right, fa_dtype o_dtype, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  fa_status s = check_varlen(cu_seqlens, B, max_seqlen, T, H, Hkv, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+  Geom g{B, H, Hkv, max_seqlen < T ? max_seqlen : T};
+  g.T = T;
+  g.cu = cu_seqlens;
+  return fwd_impl(g, q, k, v, o, lse, d, scale, window_left, window_right, o_dtype, stream);
 }
 
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
@@ -409,10 +490,32 @@ fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void*
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (ws_bytes < fa::bwd_gqa_workspace_bytes(B, H, Hkv, N, d)) return FA_ERR_INVALID_ARG;
   if ((s = check_device()) != FA_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Mask m = resolve_mask(window_left, window_right, N);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, m, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H, Hkv, N, scale, m, st);
+  return bwd_impl(Geom{B, H, Hkv, N}, q, k, v, o, lse, dO, dq, dk, dv, workspace, d, scale, window_left,
+                  window_right, stream);
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int T, int H, int Hkv, int d) {
+  if (B < 1 || check_sizes(1, H, T, d, 1.f, 0) != FA_OK || Hkv < 1 || H % Hkv != 0) return 0;
+  if ((static_cast<long long>(T) + 4LL * B + 8) * H >= (1ll << 31)) return 0;
+  return fa::bwd_varlen_workspace_bytes(B, T, H, Hkv, d);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens, void* workspace,
+                        size_t ws_bytes, int B, int max_seqlen, int T, int H, int Hkv, int d, float scale,
+                        int window_left, int window_right, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  fa_status s = check_varlen(cu_seqlens, B, max_seqlen, T, H, Hkv, d, scale);
+  if (s != FA_OK) return s;
+  if (ws_bytes < fa::bwd_varlen_workspace_bytes(B, T, H, Hkv, d)) return FA_ERR_INVALID_ARG;
+  if ((s = check_device()) != FA_OK) return s;
+  Geom g{B, H, Hkv, max_seqlen < T ? max_seqlen : T};
+  g.T = T;
+  g.cu = cu_seqlens;
+  return bwd_impl(g, q, k, v, o, lse, dO, dq, dk, dv, workspace, d, scale, window_left, window_right, stream);
 }
 
 fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -452,6 +555,8 @@ fa_status fa_get_device_error(void* stream) {
   if (word != 0u) {
     const unsigned int zero = 0u;
     if (cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    // Only malformed cu_seqlens: a caller error that the kernels clamped.
+    if (word == fa::FA_DEVERR_SEQLENS) return FA_ERR_INVALID_ARG;
     return FA_ERR_TIMEOUT;
   }
   return FA_OK;
@@ -472,8 +577,9 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Mask m = resolve_mask(-1, causal ? 0 : -1, N);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, m, st);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H, H, N, scale, m, st);
+  const Geom g{B, H, H, N};
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, scratch, g, scale, m, st);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, scratch, g, scale, m, st);
 }
 
 }  // extern "C"

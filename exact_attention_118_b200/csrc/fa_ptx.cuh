@@ -16,6 +16,7 @@ namespace fa {
 __device__ unsigned int g_device_error = 0u;
 constexpr unsigned int FA_DEVERR_TIMEOUT = 1u;
 constexpr unsigned int FA_DEVERR_SMEM_ALIGN = 2u;  // dynamic shared memory not 1 KB aligned
+constexpr unsigned int FA_DEVERR_SEQLENS = 4u;     // cu_seqlens entries outside [0, T] or not increasing
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -280,6 +281,19 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // Pack two fp32 into bf16x2 (round to nearest even): `lo` in bits 0..15.
+// Sequence b of a packed variable-length batch: its first packed row s0 and
+// its length L, from the prefix sums cu[b] and cu[b + 1]. Entries that would
+// reach outside the T packed rows, run backwards or exceed max_len are
+// clamped, so no access leaves the caller's buffers, and recorded as
+// FA_DEVERR_SEQLENS.
+__device__ __forceinline__ void seq_range(const int* cu, int b, int T, int max_len, int& s0, int& L) {
+  const int a = __ldg(cu + b), e = __ldg(cu + b + 1);
+  if ((a < 0 || e < a || e > T || e - a > max_len) && threadIdx.x == 0)
+    atomicOr(&g_device_error, FA_DEVERR_SEQLENS);
+  s0 = min(max(a, 0), T);
+  L = min(min(max(e, s0), T) - s0, max_len);
+}
+
 // Attention masks the kernels are instantiated for. Band: key j is visible
 // to query i iff i - wl <= j <= i + wr (the local window), wl, wr >= 0.
 enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskBand = 2 };

@@ -181,9 +181,48 @@ fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void*
                         int window_left, int window_right, void* stream);
 
 /*
+ * Variable-length batches (the dynamic-shape support that "FlashAttention：
+ * 优化大模型训练的内存与计算效率", cnnetsun.cn, lists among its optimisation
+ * directions): B sequences of different lengths packed back to back, with no
+ * padding. q, o, dO, dq are [T, H, d] and k, v, dk, dv [T, Hkv, d] bf16,
+ * token-major; sequence b owns packed rows [cu_seqlens[b], cu_seqlens[b+1]).
+ * lse is fp32 [H, T]. cu_seqlens is a device int32 array of B + 1
+ * non-decreasing prefix sums from 0 to at most T (4-byte aligned); every
+ * length is at most max_seqlen. Each sequence is attended on its own, with
+ * the window (causal: (-1, 0)) applied within the sequence, exactly as if it
+ * were a batch of one. The grid covers max_seqlen for every sequence; blocks
+ * past the end of a shorter sequence exit at once.
+ * Malformed cu_seqlens cannot make a kernel read or write outside the
+ * buffers: each entry is clamped to [0, T] and each length to max_seqlen, and
+ * fa_get_device_error then reports FA_ERR_INVALID_ARG. The last tile of a
+ * sequence reads the packed rows after it and masks them out; a masked
+ * product is exactly zero only for finite values, so every row of q, k, v
+ * (and of o, lse, dO for the backward) must be finite, as it is when the
+ * sequences cover all T rows (cu_seqlens[0] = 0, cu_seqlens[B] = T). The
+ * forward leaves the o and lse of rows that no sequence covers untouched; the
+ * backward's dq, dk, dv there are unspecified.
+ * The backward workspace is fa_bwd_varlen_workspace_size(B, T, H, Hkv, d)
+ * bytes (0 for invalid sizes): an fp32 [T, H, d] dQ accumulator, then two
+ * fp32 [H][S] statistics arrays with S = T + 4B + 4 rounded up to a multiple
+ * of 4 (each sequence's statistics start on a 16-byte boundary), then, when
+ * Hkv < H, two fp32 [T, Hkv, d] dK/dV accumulators; each piece rounded up to
+ * 256 bytes. Every other convention is fa_fwd_window's/fa_bwd_window's.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens, int B, int max_seqlen, int T, int H, int Hkv, int d,
+                        float scale, int window_left, int window_right, fa_dtype o_dtype, void* stream);
+size_t fa_bwd_varlen_workspace_size(int B, int T, int H, int Hkv, int d);
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                        void* workspace, size_t ws_bytes, int B, int max_seqlen, int T, int H, int Hkv,
+                        int d, float scale, int window_left, int window_right, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
- * since the last call, FA_ERR_CUDA if the synchronisation failed, else FA_OK.
+ * since the last call, FA_ERR_INVALID_ARG if the only thing recorded is a
+ * malformed cu_seqlens array (variable-length calls), FA_ERR_CUDA if the
+ * synchronisation failed, else FA_OK.
  */
 fa_status fa_get_device_error(void* stream);
 

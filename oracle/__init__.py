@@ -27,6 +27,11 @@ Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
   computation over the explicitly listed visible keys, the closed form for
   wl = wr = 0 (O = V, lse = scale q.k), unbounded windows equal to the full and
   causal masks, and central finite differences of the backward.
+- ``attention_forward_varlen`` / ``attention_backward_varlen`` packed
+  variable-length batches: each sequence attended on its own. Pinned by: a
+  pure-Python per-row computation over each row's own sequence, equal
+  lengths = the fixed-length batch, and independence from the other
+  sequences' contents.
 - ``blockwise_online_softmax_attention`` the tiled merge with running max and
   running sum. Pinned by: equality with the full-row softmax on tiny inputs,
   for several block sizes.
@@ -41,6 +46,8 @@ from .attention import (  # noqa: F401
     attention_backward_rows,
     attention_backward_gqa,
     attention_forward_gqa,
+    attention_backward_varlen,
+    attention_forward_varlen,
     band_visible,
     causal_visible,
 )

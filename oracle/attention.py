@@ -227,3 +227,47 @@ def attention_backward_gqa(q, k, v, do, scale: float, causal: bool, window=None)
     g = H // Hkv
     dq, dk, dv = attention_backward(q, _repeat_kv(k, g), _repeat_kv(v, g), do, scale, causal, window=window)
     return dq, dk.reshape(B, Hkv, g, N, -1).sum(axis=2), dv.reshape(B, Hkv, g, N, -1).sum(axis=2)
+
+
+# ------------------------------------------------------ variable-length batches
+# Packed variable-length batches (the dynamic-shape support listed among the
+# optimisation directions of "FlashAttention：优化大模型训练的内存与计算效率",
+# cnnetsun.cn): B sequences of different lengths stored back to back without
+# padding, q [T, H, d], k and v [T, H_kv, d], sequence b in rows
+# [cu[b], cu[b + 1]). Each sequence is attended on its own, as a batch of one
+# (masks apply within the sequence). lse is [H, T].
+
+def _sequence(x, a, e):
+    """Rows [a, e) of a packed [T, heads, d] array as a [1, heads, L, d] batch."""
+    return np.transpose(x[a:e], (1, 0, 2))[None]
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, scale: float, causal: bool, window=None):
+    """O [T, H, d] and lse [H, T] of packed variable-length attention. Rows no
+    sequence covers are left NaN."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    T, H, d = q.shape
+    o = np.full((T, H, v.shape[2]), np.nan)
+    lse = np.full((H, T), np.nan)
+    for a, e in zip(cu[:-1], cu[1:]):
+        if e > a:
+            ob, lb = attention_forward_gqa(_sequence(q, a, e), _sequence(k, a, e), _sequence(v, a, e), scale, causal,
+                                           window)
+            o[a:e] = np.transpose(ob[0], (1, 0, 2))
+            lse[:, a:e] = lb[0]
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_seqlens, scale: float, causal: bool, window=None):
+    """dQ [T, H, d], dK and dV [T, H_kv, d] of packed variable-length attention."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    dq, dk, dv = np.full(q.shape, np.nan), np.full(k.shape, np.nan), np.full(v.shape, np.nan)
+    for a, e in zip(cu[:-1], cu[1:]):
+        if e > a:
+            g = attention_backward_gqa(_sequence(q, a, e), _sequence(k, a, e), _sequence(v, a, e),
+                                       _sequence(do, a, e), scale, causal, window)
+            for out, gb in zip((dq, dk, dv), g):
+                out[a:e] = np.transpose(gb[0], (1, 0, 2))
+    return dq, dk, dv

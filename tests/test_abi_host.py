@@ -15,7 +15,8 @@ def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
                           "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_gqa_workspace_size",
-                          "fa_fwd_window", "fa_bwd_window",
+                          "fa_fwd_window", "fa_bwd_window", "fa_fwd_varlen", "fa_bwd_varlen",
+                          "fa_bwd_varlen_workspace_size",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
                           "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
@@ -164,3 +165,33 @@ def test_window_calls_reject_bad_arguments():
     need = fa.fa_bwd_gqa_workspace_size(1, 8, 2, 256, 64)
     assert fa.fa_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 1, 8, 2, 256, 64,
                             0.1, 16, 16, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_varlen_workspace_size_formula():
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for B, T, H, Hkv, d in ((3, 1000, 8, 8, 64), (7, 4097, 16, 4, 128)):
+        S = (T + 4 * B + 4 + 3) // 4 * 4
+        want = up(T * H * d * 4) + 2 * up(H * S * 4) + (2 * up(T * Hkv * d * 4) if Hkv < H else 0)
+        assert fa.fa_bwd_varlen_workspace_size(B, T, H, Hkv, d) == want
+    assert fa.fa_bwd_varlen_workspace_size(2, 100, 8, 3, 64) == 0
+    assert fa.fa_bwd_varlen_workspace_size(0, 100, 8, 8, 64) == 0
+
+
+def test_varlen_calls_reject_bad_arguments():
+    ok = dict(B=2, max_seqlen=64, T=100, H=4, Hkv=2, d=64)
+
+    def fwd(cu=FAKE, **kw):
+        a = {**ok, **kw}
+        return fa.fa_fwd_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu, a["B"], a["max_seqlen"], a["T"], a["H"], a["Hkv"],
+                                a["d"], 0.1, -1, 0, fa.FA_BF16, None)
+
+    assert fwd(cu=None) == fa.FA_ERR_INVALID_ARG
+    assert fwd(cu=FAKE + 2) == fa.FA_ERR_INVALID_ARG  # cu_seqlens not 4-byte aligned
+    assert fwd(B=0) == fa.FA_ERR_INVALID_ARG
+    assert fwd(max_seqlen=0) == fa.FA_ERR_INVALID_ARG
+    assert fwd(T=0) == fa.FA_ERR_INVALID_ARG
+    assert fwd(Hkv=3) == fa.FA_ERR_INVALID_ARG
+    assert fwd(d=80) == fa.FA_ERR_UNSUPPORTED
+    need = fa.fa_bwd_varlen_workspace_size(2, 100, 4, 2, 64)
+    assert fa.fa_bwd_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 2, 64, 100,
+                            4, 2, 64, 0.1, -1, 0, None) == fa.FA_ERR_INVALID_ARG

@@ -415,3 +415,59 @@ def test_window_backward_central_finite_differences(wl, wr):
         else:
             err = np.max(np.abs(num - g)) / np.max(np.abs(g))
             assert err <= 1e-6, (which, err)
+
+
+# ------------------------------------------------------ variable-length batches
+
+def test_varlen_against_per_row_python():
+    """Three packed sequences (one empty), causal and full: every row against
+    a plain-Python softmax over the keys of its own sequence only."""
+    from oracle import attention_forward_varlen
+
+    cu = [0, 4, 4, 11, 13]
+    T, H, d = 13, 2, 3
+    q, k, v = (_rand((T, H, d), s) for s in (101, 102, 103))
+    for causal in (False, True):
+        o, lse = attention_forward_varlen(q, k, v, np.array(cu), 0.8, causal)
+        for a, e in zip(cu[:-1], cu[1:]):
+            for i in range(a, e):
+                for h in range(H):
+                    keys = range(a, i + 1) if causal else range(a, e)
+                    x = [0.8 * sum(q[i, h, c] * k[j, h, c] for c in range(d)) for j in keys]
+                    mx = max(x)
+                    w = [math.exp(t - mx) for t in x]
+                    ref = [sum(wt * v[j, h, c] for wt, j in zip(w, keys)) / sum(w) for c in range(d)]
+                    assert np.allclose(o[i, h], ref, rtol=0, atol=1e-13)
+                    assert abs(lse[h, i] - (mx + math.log(sum(w)))) < 1e-13
+
+
+def test_varlen_equal_lengths_is_the_fixed_batch():
+    from oracle import attention_backward_varlen, attention_forward_varlen
+
+    B, H, N, d = 3, 2, 10, 4
+    q, k, v, do = (_rand((B, H, N, d), s) for s in (111, 112, 113, 114))
+    packed = lambda x: np.transpose(x, (0, 2, 1, 3)).reshape(B * N, H, d)  # noqa: E731
+    cu = np.arange(B + 1) * N
+    for causal in (False, True):
+        o, lse = attention_forward_varlen(packed(q), packed(k), packed(v), cu, 0.5, causal)
+        o_ref, lse_ref = attention_forward(q, k, v, 0.5, causal)
+        assert np.array_equal(o, packed(o_ref))
+        assert np.array_equal(lse, np.transpose(lse_ref, (1, 0, 2)).reshape(H, B * N))
+        g = attention_backward_varlen(packed(q), packed(k), packed(v), packed(do), cu, 0.5, causal)
+        g_ref = attention_backward(q, k, v, do, 0.5, causal)
+        for a, b in zip(g, g_ref):
+            assert np.array_equal(a, packed(b))
+
+
+def test_varlen_sequences_are_independent():
+    from oracle import attention_forward_varlen
+
+    cu = np.array([0, 5, 12, 20])
+    q, k, v = (_rand((20, 2, 4), s) for s in (121, 122, 123))
+    o, _ = attention_forward_varlen(q, k, v, cu, 0.7, False)
+    k2, v2 = k.copy(), v.copy()
+    k2[5:12] += 3.0
+    v2[5:12] -= 1.0
+    o2, _ = attention_forward_varlen(q, k2, v2, cu, 0.7, False)
+    assert np.array_equal(o[:5], o2[:5]) and np.array_equal(o[12:], o2[12:])
+    assert not np.allclose(o[5:12], o2[5:12])

@@ -100,3 +100,25 @@ def make_workload_inputs(w: Workload, with_grad_out: Optional[bool] = None):
     if with_grad_out is None:
         with_grad_out = w.backward
     return make_inputs(w.B, w.H, w.N, w.d, w.seed, w.qk_std, with_grad_out)
+
+
+def make_varlen_inputs(lengths, H: int, Hkv: int, d: int, seed: int, qk_std: float = 1.0):
+    """A packed variable-length batch: sequences of the given lengths stored
+    back to back. Returns a dict with ``q`` and ``do`` [T, H, d], ``k`` and ``v``
+    [T, Hkv, d] (bf16 CPU tensors, drawn in that order from one seeded
+    generator) and ``cu_seqlens`` (int32 [B + 1] prefix sums)."""
+    lengths = [int(n) for n in lengths]
+    T = sum(lengths)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    out = {}
+    for name in ("q", "k", "v", "do"):
+        t = torch.randn((T, Hkv if name in ("k", "v") else H, d), generator=g, dtype=torch.float32)
+        if name in ("q", "k") and qk_std != 1.0:
+            t.mul_(qk_std)
+        out[name] = t.to(torch.bfloat16)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
+    return out
