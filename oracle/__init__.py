@@ -32,6 +32,12 @@ Functions and what pins them (the pins live in ``tests/test_oracle_*.py``):
   pure-Python per-row computation over each row's own sequence, equal
   lengths = the fixed-length batch, and independence from the other
   sequences' contents.
+- ``e4m3_decode`` the 8-bit e4m3 code to value map, written from the format
+  definition. Pinned by: torch's float8_e4m3fn for all 256 codes and
+  hand-worked codes (448, 2^-6, 2^-9, NaN).
+- ``attention_forward_fp8`` exact attention of per-tensor-scaled e4m3 Q, K,
+  V. Pinned by: the decoder's pins, the trade between a tensor's scale and the
+  softmax scale, linearity of O in the V scale, and lse's independence of it.
 - ``blockwise_online_softmax_attention`` the tiled merge with running max and
   running sum. Pinned by: equality with the full-row softmax on tiny inputs,
   for several block sizes.
@@ -51,4 +57,5 @@ from .attention import (  # noqa: F401
     band_visible,
     causal_visible,
 )
+from .fp8 import attention_forward_fp8, e4m3_decode  # noqa: F401
 from .online_softmax import blockwise_online_softmax_attention  # noqa: F401

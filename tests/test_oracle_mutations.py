@@ -169,3 +169,31 @@ def test_window_off_by_one_is_caught(monkeypatch, side):
 
     monkeypatch.setattr(att, "band_visible", bad)
     assert not _window_ok()
+
+
+def _e4m3_ok(decode):
+    import torch
+
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = decode(codes.numpy())
+    return bool(np.all((np.isnan(ref) & np.isnan(got)) | (ref == got)))
+
+
+@pytest.mark.parametrize("mistake", ["bias8", "no_subnormal", "mantissa_over_16"])
+def test_e4m3_decoder_mistakes_are_caught(mistake):
+    import oracle.fp8 as f8
+
+    assert _e4m3_ok(f8.e4m3_decode)
+
+    def bad(codes):
+        c = np.asarray(codes).astype(np.int64) & 0xFF
+        s = np.where(c & 0x80, -1.0, 1.0)
+        e, m = (c >> 3) & 0xF, (c & 7).astype(np.float64)
+        bias, div = (8.0 if mistake == "bias8" else 7.0), (16.0 if mistake == "mantissa_over_16" else 8.0)
+        norm = (1.0 + m / div) * np.exp2(e - bias)
+        sub = norm if mistake == "no_subnormal" else m / div * 2.0 ** (1 - bias)
+        v = np.where(e == 0, sub, norm)
+        return s * np.where((e == 15) & ((c & 7) == 7), np.nan, v)
+
+    assert not _e4m3_ok(bad)

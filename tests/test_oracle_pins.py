@@ -471,3 +471,53 @@ def test_varlen_sequences_are_independent():
     o2, _ = attention_forward_varlen(q, k2, v2, cu, 0.7, False)
     assert np.array_equal(o[:5], o2[:5]) and np.array_equal(o[12:], o2[12:])
     assert not np.allclose(o[5:12], o2[5:12])
+
+
+# ------------------------------------------------------------ FP8 (e4m3) inputs
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    from oracle import e4m3_decode
+
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = e4m3_decode(codes.numpy())
+    both_nan = np.isnan(ref) & np.isnan(got)
+    assert np.all(both_nan | (ref == got))
+    assert np.sum(np.isnan(got)) == 2  # 0x7F and 0xFF
+
+
+def test_e4m3_decode_hand_values():
+    from oracle import e4m3_decode
+
+    table = {0x00: 0.0, 0x80: -0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+             0x39: 1.125, 0xB8: -1.0, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0, 0x77: 240.0, 0x30: 0.5}
+    for c, want in table.items():
+        assert e4m3_decode(np.array([c]))[0] == want, hex(c)
+    assert np.isnan(e4m3_decode(np.array([0x7F]))[0])
+
+
+def _fp8_case(seed, n=40, d=16):
+    g = np.random.default_rng(seed)
+    return [g.integers(0, 256, (1, 2, n, d)) for _ in range(3)]
+
+
+def _finite(codes):
+    return np.where((codes & 0x7F) == 0x7F, 0x38, codes)  # replace NaN codes by 1.0
+
+
+def test_fp8_scale_trades_with_softmax_scale():
+    from oracle import attention_forward_fp8
+
+    q8, k8, v8 = (_finite(c) for c in _fp8_case(131))
+    o1, l1 = attention_forward_fp8(q8, k8, v8, 0.01, 0.02, 0.5, 0.125, True)
+    o2, l2 = attention_forward_fp8(q8, k8, v8, 0.02, 0.04, 0.5, 0.125 / 4, True)
+    assert np.allclose(o1, o2, rtol=1e-13, atol=1e-15) and np.allclose(l1, l2, rtol=1e-13, atol=1e-13)
+
+
+def test_fp8_v_scale_is_linear_and_leaves_lse():
+    from oracle import attention_forward_fp8
+
+    q8, k8, v8 = (_finite(c) for c in _fp8_case(132))
+    o1, l1 = attention_forward_fp8(q8, k8, v8, 0.01, 0.02, 0.5, 0.125, False)
+    o2, l2 = attention_forward_fp8(q8, k8, v8, 0.01, 0.02, 1.5, 0.125, False)
+    assert np.allclose(o2, 3.0 * o1, rtol=1e-13, atol=1e-15) and np.array_equal(l1, l2)

@@ -122,3 +122,23 @@ def make_varlen_inputs(lengths, H: int, Hkv: int, d: int, seed: int, qk_std: flo
         cu.append(cu[-1] + n)
     out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
     return out
+
+
+def make_fp8_inputs(B: int, H: int, N: int, d: int, seed: int, kv_heads: Optional[int] = None):
+    """Q, K, V as e4m3 codes with per-tensor dequantisation scales.
+
+    Draws standard-normal fp32 Q, K, V (K, V with ``kv_heads`` heads if set)
+    from one seeded generator, picks each tensor's scale as its largest
+    magnitude / 448 (the largest finite e4m3 value), and rounds x / scale to
+    e4m3 with torch's float8_e4m3fn cast. Returns a dict with uint8 tensors
+    ``q8``, ``k8``, ``v8`` and floats ``q_scale``, ``k_scale``, ``v_scale``."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    Hkv = H if kv_heads is None else int(kv_heads)
+    out = {}
+    for name, heads in (("q", H), ("k", Hkv), ("v", Hkv)):
+        t = torch.randn((B, heads, N, d), generator=g, dtype=torch.float32)
+        s = float(t.abs().max()) / 448.0
+        out[name + "8"] = (t / s).to(torch.float8_e4m3fn).view(torch.uint8)
+        out[name + "_scale"] = s
+    return out
