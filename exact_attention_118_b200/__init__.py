@@ -35,6 +35,7 @@ _SIGNATURES = {
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_gqa_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _F, _F, _I, _I, _I, _P]),
     "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "fa_bwd_varlen_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "fa_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _I, _F,
@@ -101,6 +102,12 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, B, H, N, d, sca
 
 def fa_bwd_gqa_workspace_size(B, H, Hkv, N, d) -> int:
     return _lib.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d)
+
+
+def fa_fwd_fp8(q8, k8, v8, o, lse, B, H, Hkv, N, d, scale, q_scale, k_scale, v_scale, window_left, window_right,
+               o_dtype, stream) -> int:
+    return _lib.fa_fwd_fp8(q8, k8, v8, o, lse, B, H, Hkv, N, d, scale, q_scale, k_scale, v_scale, window_left,
+                           window_right, o_dtype, stream)
 
 
 def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, max_seqlen, T, H, Hkv, d, scale, window_left, window_right,

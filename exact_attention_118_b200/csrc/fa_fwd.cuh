@@ -36,6 +36,12 @@
 //   the result is the same because O and l share the same stale m, and the
 //   largest p is at most 2^8);  p_ij = 2^(lambda*S_ij - m);  l = alpha*l + sum p.
 //   Epilogue: O /= l;  lse = ln2 * (m + log2 l).
+//
+// FP8 (FP8 = true, D = 128): Q, K, V are e4m3 codes with per-tensor
+// dequantisation scales. S and PV run as kind::f8f6f4 MMAs (K = 32 per
+// instruction); the Q and K scales fold into lambda and the V scale into the
+// epilogue (o_scale). P is rounded to e4m3 for the PV product (p <= 2^8 < 448,
+// the largest e4m3 value); l sums the unrounded p.
 #pragma once
 #include <cuda.h>
 #include "fa_ptx.cuh"
@@ -50,16 +56,19 @@ struct FwdParams {
   int Hkv;  // K/V heads (H % Hkv == 0; query head h reads K/V head h / (H / Hkv))
   int N;
   int n_pairs;       // ceil(N / 256): CTAs per (batch, head)
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (FP8: times the Q and K dequantisation scales)
+  float o_scale;     // multiplies O in the epilogue: 1, or the V dequantisation scale (FP8)
   int wl, wr;        // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
   const int* cu_seqlens;  // packed variable length: [B + 1] prefix sums of the lengths; else nullptr
   int T;                  // packed rows (variable length only); N is then the longest length
 };
 
-template <int D>
+template <int D, int ESZ = 2>  // ESZ: bytes per element (2 bf16, 1 e4m3)
 struct FwdLayout {
-  static constexpr int kTile = 128 * D * 2;          // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kRowBytes = D * ESZ;
+  static constexpr int kTile = 128 * kRowBytes;               // one 128-row tile
+  static constexpr int kChunks = kRowBytes / 128;             // 128-byte column chunks per row
+  static constexpr int kStages = (kRowBytes == 256) ? 2 : 4;  // K/V ring depth
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTile;
   static constexpr int kK = 2 * kTile;
@@ -73,13 +82,16 @@ struct FwdLayout {
 constexpr int kFwdThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D, int MASK, bool OF32>
+template <int D, int MASK, bool OF32, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D>;
+  static_assert(!FP8 || D == 128, "the FP8 forward is built for D = 128");
+  constexpr int ESZ = FP8 ? 1 : 2;
+  using L = FwdLayout<D, ESZ>;
+  constexpr int CW = 128 / ESZ;  // elements per 128-byte chunk
   constexpr int S = L::kStages;
-  constexpr int KCH = D / 64;  // 64-column (128-byte) chunks per row
+  constexpr int KCH = L::kChunks;  // 128-byte column chunks per row
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -176,19 +188,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_arrive_expect_tx(q_full, 2 * L::kTile);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * 64, s0 + q0 + 128 * t, hq);
+          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * CW, s0 + q0 + 128 * t, hq);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < J; ++j) {
         const int s = j % S, u = j / S;
         if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(k_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * 64, s0 + (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * CW, s0 + (j0 + j) * 128, bkv);
         k_issued = j + 1;
         if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + s, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * 64, s0 + (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * CW, s0 + (j0 + j) * 128, bkv);
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.
@@ -199,27 +211,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);  // Q, K both K-major
-      constexpr uint32_t kIdO = idesc_bf16(128, D, 0, 1);    // P (TMEM), V MN-major
+      // S: Q, K both K-major. PV: P from TMEM, V MN-major.
+      constexpr uint32_t kIdS = FP8 ? idesc_e4m3(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t kIdO = FP8 ? idesc_e4m3(128, D, 0, 1) : idesc_bf16(128, D, 0, 1);
       const uint32_t q_addr[2] = {smem_u32(smem + L::kQ0), smem_u32(smem + L::kQ1)};
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
 
       auto issue_s = [&](int t, int stage) {
         const uint32_t ka = k_addr + stage * L::kTile;
+        // Each MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3).
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(q_addr[t] + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdS,
-                 kk > 0);
+          const uint64_t da = sdesc_sw128(q_addr[t] + off, 16, 1024), db = sdesc_sw128(ka + off, 16, 1024);
+          if (FP8)
+            mma_ss_f8(tmem + t * 128, da, db, kIdS, kk > 0);
+          else
+            mma_ss(tmem + t * 128, da, db, kIdS, kk > 0);
         }
       };
       auto issue_pv = [&](int t, int stage, bool acc) {
         const uint32_t va = v_addr + stage * L::kTile;
+        // Each MMA takes 32 bytes of P per row (8 TMEM columns: 16 bf16 or 32
+        // e4m3 keys) and the matching 16 or 32 rows of V.
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), kIdO,
-                 (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4 * ESZ; ++kk) {
+          const uint64_t dv = sdesc_sw128(va + kk * (32 / ESZ) * 128, 16384, 1024);
+          if (FP8)
+            mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, dv, kIdO, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, dv, kIdO, (acc || kk > 0) ? 1u : 0u);
         }
       };
 
@@ -331,17 +353,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float neg_m = (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m;
       float rs0 = 0.f, rs1 = 0.f;
       uint32_t pk[64];
+      if (FP8) {
+        // Four e4m3 probabilities per TMEM column: P fills 32 columns.
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(fmaf(s[2 * c], lam, neg_m));
-        const float p1 = ex2(fmaf(s[2 * c + 1], lam, neg_m));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c] = pack_bf16(p0, p1);
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2(fmaf(s[4 * c], lam, neg_m));
+          const float p1 = ex2(fmaf(s[4 * c + 1], lam, neg_m));
+          const float p2 = ex2(fmaf(s[4 * c + 2], lam, neg_m));
+          const float p3 = ex2(fmaf(s[4 * c + 3], lam, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          rs0 += p2;
+          rs1 += p3;
+          pk[c] = pack_e4m3x4(p0, p1, p2, p3);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2(fmaf(s[2 * c], lam, neg_m));
+          const float p1 = ex2(fmaf(s[2 * c + 1], lam, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          pk[c] = pack_bf16(p0, p1);
+        }
       }
       l = l * alpha + (rs0 + rs1);
       tmem_st32(tS + 0, pk + 0);
-      tmem_st32(tS + 32, pk + 32);
+      if (!FP8) tmem_st32(tS + 32, pk + 32);
       if (j > 0) {
         // PV_{j-1} finished before S_j (same issuing thread, committed
         // earlier), so this wait is immediate; it keeps the phase count exact.
@@ -370,7 +408,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (nt - 1) & 1, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = (FP8 ? p.o_scale : 1.f) / l;
         const bool valid = qi < N;
         const int qv = valid ? qi : 0;
         // O row (units of D elements) and lse index of query qi.

@@ -145,11 +145,11 @@ Mask resolve_mask(int wl, int wr, int N) {
   return {fa::kMaskBand, l, r};
 }
 
-template <int D, int MASK, bool OF32>
+template <int D, int MASK, bool OF32, bool FP8 = false>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
                      cudaStream_t st) {
-  auto kern = fa::fa_fwd_kernel<D, MASK, OF32>;
-  const int smem = fa::FwdLayout<D>::kAlloc;
+  auto kern = fa::fa_fwd_kernel<D, MASK, OF32, FP8>;
+  const int smem = fa::FwdLayout<D, FP8 ? 1 : 2>::kAlloc;
   if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
     return cuda_fail(e);
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
@@ -157,12 +157,12 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return launch_status();
 }
 
-template <int D, bool OF32>
+template <int D, bool OF32, bool FP8 = false>
 fa_status launch_fwd_mask(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const fa::FwdParams& p, int mode, cudaStream_t st) {
-  if (mode == fa::kMaskCausal) return launch_fwd<D, fa::kMaskCausal, OF32>(tq, tk, tv, p, st);
-  if (mode == fa::kMaskBand) return launch_fwd<D, fa::kMaskBand, OF32>(tq, tk, tv, p, st);
-  return launch_fwd<D, fa::kMaskNone, OF32>(tq, tk, tv, p, st);
+  if (mode == fa::kMaskCausal) return launch_fwd<D, fa::kMaskCausal, OF32, FP8>(tq, tk, tv, p, st);
+  if (mode == fa::kMaskBand) return launch_fwd<D, fa::kMaskBand, OF32, FP8>(tq, tk, tv, p, st);
+  return launch_fwd<D, fa::kMaskNone, OF32, FP8>(tq, tk, tv, p, st);
 }
 
 // 2-D fp32 map of a [BH][Np] statistics array (Np >= N, a multiple of 4),
@@ -375,6 +375,7 @@ fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, v
   p.N = g.N;
   p.n_pairs = (g.N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_scale = 1.f;
   const Mask m = resolve_mask(window_left, window_right, g.N);
   p.wl = m.wl;
   p.wr = m.wr;
@@ -387,6 +388,36 @@ fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, v
                : launch_fwd_mask<64, false>(tq, tk, tv, p, m.mode, st);
   return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, p, m.mode, st)
              : launch_fwd_mask<128, false>(tq, tk, tv, p, m.mode, st);
+}
+
+// The FP8 forward (fixed-length layout, D = 128); arguments already checked.
+fa_status fwd_fp8_impl(const Geom& g, const void* q8, const void* k8, const void* v8, void* o, float* lse,
+                       float scale, float q_scale, float k_scale, float v_scale, int window_left, int window_right,
+                       fa_dtype o_dtype, void* stream) {
+  fa_status s;
+  alignas(64) CUtensorMap tq, tk, tv;
+  const auto u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if ((s = make_head_map(&tq, q8, g, g.H, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
+  if ((s = make_head_map(&tk, k8, g, g.Hkv, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
+  if ((s = make_head_map(&tv, v8, g, g.Hkv, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.BH = g.B * g.H;
+  p.H = g.H;
+  p.Hkv = g.Hkv;
+  p.N = g.N;
+  p.n_pairs = (g.N + 255) / 256;
+  p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  p.o_scale = v_scale;
+  const Mask m = resolve_mask(window_left, window_right, g.N);
+  p.wl = m.wl;
+  p.wr = m.wr;
+  p.cu_seqlens = g.cu;
+  p.T = g.T;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return o_dtype == FA_F32 ? launch_fwd_mask<128, true, true>(tq, tk, tv, p, m.mode, st)
+                           : launch_fwd_mask<128, false, true>(tq, tk, tv, p, m.mode, st);
 }
 
 // The backward for either layout; arguments already checked.
@@ -455,6 +486,23 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   g.T = T;
   g.cu = cu_seqlens;
   return fwd_impl(g, q, k, v, o, lse, d, scale, window_left, window_right, o_dtype, stream);
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H, int Hkv,
+                     int N, int d, float scale, float q_scale, float k_scale, float v_scale, int window_left,
+                     int window_right, fa_dtype o_dtype, void* stream) {
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  fa_status s = check_sizes(B, H, N, d, scale, 0);
+  if (s != FA_OK) return s;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  for (float x : {q_scale, k_scale, v_scale})
+    if (!(std::isfinite(x) && x > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if ((s = check_device()) != FA_OK) return s;
+  return fwd_fp8_impl(Geom{B, H, Hkv, N}, q8, k8, v8, o, lse, scale, q_scale, k_scale, v_scale, window_left,
+                      window_right, o_dtype, stream);
 }
 
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,

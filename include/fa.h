@@ -218,6 +218,26 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         int d, float scale, int window_left, int window_right, void* stream);
 
 /*
+ * FP8 forward (low-precision inputs, listed among the optimisation directions
+ * of "FlashAttention：优化大模型训练的内存与计算效率", cnnetsun.cn). q8 is
+ * [B, H, N, 128], k8 and v8 [B, Hkv, N, 128], all 8-bit e4m3 codes (sign,
+ * 4-bit exponent with bias 7, 3-bit mantissa; no infinities), each tensor with
+ * one fp32 dequantisation scale: the value of a code c of Q is
+ * e4m3(c) * q_scale, and likewise for K and V. Computes the attention of the
+ * dequantised tensors with the window convention of fa_fwd_window, writing O
+ * (bf16 or fp32, [B, H, N, 128]) and lse (fp32 [B, H, N]). Both products run
+ * on the tensor cores in e4m3 with fp32 accumulation; the probabilities are
+ * rounded to e4m3 (relative error at most 2^-4, absolute at most 2^-10 below
+ * 2^-6) before they multiply V, and lse uses the unrounded row sums. d must be
+ * 128 (else FA_ERR_UNSUPPORTED); a scale that is not finite and positive gives
+ * FA_ERR_INVALID_ARG. There is no FP8 backward.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse,
+                     int B, int H, int Hkv, int N, int d, float scale,
+                     float q_scale, float k_scale, float v_scale,
+                     int window_left, int window_right, fa_dtype o_dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word.
  * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
  * since the last call, FA_ERR_INVALID_ARG if the only thing recorded is a

@@ -16,7 +16,7 @@ def test_library_loads_and_exports_every_header_symbol():
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
                           "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_gqa_workspace_size",
                           "fa_fwd_window", "fa_bwd_window", "fa_fwd_varlen", "fa_bwd_varlen",
-                          "fa_bwd_varlen_workspace_size",
+                          "fa_bwd_varlen_workspace_size", "fa_fwd_fp8",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
                           "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
@@ -195,3 +195,15 @@ def test_varlen_calls_reject_bad_arguments():
     need = fa.fa_bwd_varlen_workspace_size(2, 100, 4, 2, 64)
     assert fa.fa_bwd_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 2, 64, 100,
                             4, 2, 64, 0.1, -1, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fp8_forward_rejects_bad_arguments():
+    def call(d=128, qs=1.0, ks=1.0, vs=1.0, Hkv=2):
+        return fa.fa_fwd_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, Hkv, 256, d, 0.1, qs, ks, vs, -1, 0, fa.FA_BF16, None)
+
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(qs=0.0) == fa.FA_ERR_INVALID_ARG
+    assert call(ks=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert call(vs=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert call(vs=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert call(Hkv=3) == fa.FA_ERR_INVALID_ARG
