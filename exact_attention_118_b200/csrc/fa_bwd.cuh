@@ -29,7 +29,7 @@
 // own elementwise warpgroup, so the two groups overlap each other's waits.
 //
 // Roles (512 threads): warp 0 TMA producer (Q, dO, lse2 and D tiles), warps 1
-// and 2 MMA issuers, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
+// to 3 MMA issuers, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
 // dQ^T), warps 8-11 and 12-15 two elementwise warpgroups (thread = key row)
 // that take alternate query tiles.
 #pragma once
@@ -227,17 +227,20 @@ template <int D>
 struct BwdLayout {
   static constexpr int kKV = 128 * D * 2;  // K or V tile: 128 keys
   static constexpr int kQT = 64 * D * 2;   // Q or dO tile: 64 queries
-  static constexpr int kStages = 4;        // Q/dO/lse2/D ring depth
+  static constexpr int kStages = (D == 128) ? 3 : 4;  // Q/dO/lse2/D ring depth
   static constexpr int kDSTile = 128 * 64 * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kKV;
   static constexpr int kQ = 2 * kKV;
   static constexpr int kDO = kQ + kStages * kQT;
-  // [2] dS tiles [128 keys][64 queries]; after the dQ MMA has read tile b it
-  // doubles as the fp32 staging area for dQ_i (two halves of 32 queries).
+  // [2] dS tiles [128 keys][64 queries].
   static constexpr int kDS = kDO + kStages * kQT;
   static constexpr int kStat = kDS + 2 * kDSTile;  // [kStages] x {lse2[64], D[64]}
-  static constexpr int kBar = kStat + kStages * 512;
+  // [2] fp32 staging halves for dQ_i (32 queries x D each), so one half is
+  // written while the TMA engine still reads the other.
+  static constexpr int kStgHalf = 32 * D * 4;
+  static constexpr int kStg = (kStat + kStages * 512 + 1023) & ~1023;
+  static constexpr int kBar = kStg + 2 * kStgHalf;
   static constexpr int kBytes = kBar + 256;
   // The kernel checks that the dynamic shared memory base is 1 KB aligned
   // (it is: the window starts on a 1 KB boundary) instead of reserving slack.
@@ -245,8 +248,8 @@ struct BwdLayout {
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-// Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warps 1
-// and 2 MMA issuers, warp 1 also TMEM owner, warp 3 idle), 4-7 dQ drain, 8-11 elementwise
+// Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warps 1-3
+// MMA issuers, warp 1 also TMEM owner), 4-7 dQ drain, 8-11 elementwise
 // (even iterations, TMEM buffer 0), 12-15 elementwise (odd iterations, buffer
 // 1). Launched at 128 registers per thread (512 x 128 = the 64K register
 // file; each SM sub-partition holds one warp of every warpgroup); the groups
@@ -285,8 +288,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_full = p_full + 2;       // [2]
   uint64_t* dq_full = ds_full + 2;      // [2]
   uint64_t* dq_empty = dq_full + 2;     // [2]
-  uint64_t* stg_free = dq_empty + 2;    // [2] dS tile b free again (dQ staging read)
-  uint64_t* y_done = stg_free + 2;      // [2] dV/dK of the buffer's last iteration done
+  uint64_t* y_done = dq_empty + 2;      // [2] dK of the buffer's last iteration done
   uint64_t* acc_full = y_done + 2;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -347,11 +349,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(ds_full + b, 4);
       mbar_init(dq_full + b, 1);
       mbar_init(dq_empty + b, 4);
-      mbar_init(stg_free + b, 1);
       mbar_init(y_done + b, 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(mma_done, 2);
+    mbar_init(acc_full, 2);   // last dV (X) and last dK (Y)
+    mbar_init(mma_done, 3);   // one per MMA issuer
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -399,16 +400,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_parity_drain(kv_full, 0);
       for (int it = max(0, issued - QS); it < issued; ++it) wait_parity_drain(qd_full + it % QS, (it / QS) & 1);
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp >= 1 && warp <= 3) {
     // ------------------------------------------------------- MMA issuers
-    // One issuing thread cannot keep the tensor core busy with these MMA
-    // shapes, so two share the work: X (warp 1) issues S^T and dQ^T, Y (warp
-    // 2) issues dP^T, dV and dK. They meet at TMEM buffer S[b]: S^T(it+2) may
-    // overwrite it only after Y's dV(it)/dK(it) have read P^T/dS^T from it
-    // (barrier y_done[b]). Both read the Q/dO stage, so qd_empty takes one
-    // release from each.
+    // Issuing one tcgen05.mma costs the issuing thread about 100 cycles
+    // (measured), longer than a 128 x 64 x 16 product takes on the tensor
+    // core, so three threads share the 32 instructions of an iteration:
+    // X (warp 1) issues S^T and dV, Y (warp 2) dP^T and dK, Z (warp 3) dQ^T.
+    // X and Y meet at TMEM buffer S[b]: S^T(it+2) may overwrite it only after
+    // dK(it) has read dS^T from it (barrier y_done[b]; dV(it) is X's own and
+    // runs first). X and Y read the Q/dO stage, so qd_empty takes one release
+    // from each.
     if (lane == 0) {
-      const bool is_x = (warp == 1);
+      const bool is_x = (warp == 1), is_z = (warp == 3);
       constexpr uint32_t kIdST = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T: K-major A and B
       constexpr uint32_t kIdAcc = idesc_bf16(128, D, 0, 1);  // dV, dK: A TMEM, B MN-major
       constexpr uint32_t kIdDQ = idesc_bf16(D, 64, 1, 1);    // dQ^T: A, B MN-major
@@ -442,13 +445,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  sdesc_sw128(ds_addr + b * L::kDSTile + kk * 2048, 8192, 1024), kIdDQ, kk > 0);
       };
 
-      bool ok = wait_parity(kv_full, 0, abort_flag) && wait_parity(qd_full, 0, abort_flag);
-      if (ok) {
+      bool ok = wait_parity(kv_full, 0, abort_flag) && (is_z || wait_parity(qd_full, 0, abort_flag));
+      if (ok && !is_z) {
         tc_fence_after();
         if (is_x) {
           issue_t(0, k_addr, q_addr);
           mma_commit(s_full + 0);
-          mma_commit(qd_empty + 0);
         } else {
           issue_t(128, v_addr, do_addr);
           mma_commit(dp_full + 0);
@@ -458,23 +460,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int b = it & 1, s = it % QS;
         const int nb = b ^ 1, ns = (it + 1) % QS;
         const bool has_next = it + 1 < n_it;
-        if (is_x) {
+        if (is_z) {
+          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_dq(b);
+          mma_commit(dq_full + b);
+        } else if (is_x) {
           if (has_next) {
             if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
             if (it >= 1 && !(ok = wait_parity(y_done + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
             tc_fence_after();
             issue_t(64 * nb, k_addr, q_addr + ns * L::kQT);
             mma_commit(s_full + nb);
-            mma_commit(qd_empty + ns);
           }
-          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_dq(b);
-          mma_commit(dq_full + b);
-        } else {
           if (!(ok = wait_parity(p_full + b, (it >> 1) & 1, abort_flag))) break;
           tc_fence_after();
           issue_acc(t_dv, 64 * b, do_addr + s * L::kQT, it > 0);
+          mma_commit(qd_empty + s);
+        } else {
           if (has_next) {
             if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
             if (it >= 1 && !(ok = wait_parity(dq_empty + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
@@ -489,8 +492,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit(qd_empty + s);
         }
       }
-      if (ok && !is_x) mma_commit(acc_full);
-      // Let every MMA both issuers started finish before TMEM is freed.
+      if (ok && !is_z) mma_commit(acc_full);
+      // Let every MMA the issuers started finish before TMEM is freed.
       mma_commit(mma_done);
       wait_parity_drain(mma_done, 0);
     }
@@ -556,9 +559,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b);
 
-      // dS tile b was last used for staging dQ of iteration it - 2.
-      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag) &&
-                                       (it < 2 || wait_parity(stg_free + b, ((it - 2) >> 1) & 1, abort_flag)));
+      // dS tile b was last read by dQ^T(it - 2), which finished before the
+      // drain released its TMEM buffer and so before dP^T(it) was issued.
+      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -631,10 +634,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (wg == 1) {
     // ------------------------------------------------- dQ drain (warps 4-7)
     // dQ_i^T sits in TMEM with the head-dim index on lanes and the 64 queries
-    // on columns. The drain copies it to the dS tile b (free once the dQ MMA
-    // that read it is done) as an fp32 [32 queries][D] half-tile, and one TMA
-    // reduce-add per half adds it into the fp32 accumulator; the TMA engine
-    // streams the reduction to L2 while the warps move on.
+    // on columns. The drain copies each half (32 queries) into its own fp32
+    // [32][D] staging buffer and one TMA reduce-add per half adds it into the
+    // fp32 accumulator; the TMA engine streams the reduction to L2 while the
+    // warps stage the next half, waiting only for that buffer's previous read.
     setmaxnreg_dec<kRegDrain>();
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -658,11 +661,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_empty + b);
       }
-      float* stg = reinterpret_cast<float*>(smem + L::kDS + b * L::kDSTile);
       const int q0 = q_start(it), bhq = q_head(it);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (h == 1 && leader) bulk_wait_group_read0();  // half 0 has been read
+        float* stg = reinterpret_cast<float*>(smem + L::kStg + h * L::kStgHalf);
+        // Groups go out in order (it-1, 0), (it-1, 1), (it, 0), ...: at most one
+        // pending means the previous read of this half's buffer is done.
+        if (leader) bulk_wait_group_read1();
         named_bar_sync(1, 128);
         if (ok && holds) {
 #pragma unroll
@@ -674,10 +679,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_reduce_add_3d(&tm_dq, stg, 0, s0 + q0 + 32 * h, bhq);
           bulk_commit_group();
         }
-      }
-      if (leader) {
-        bulk_wait_group_read0();
-        if (ok) mbar_arrive(stg_free + b);
       }
     }
     if (leader) bulk_wait_group0();
