@@ -44,10 +44,10 @@ WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then caus
 
 # DRAM traffic of one non-causal main backward launch of the workload above:
 # dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the same
-# kernel at H=4 (124.7 MB), scaled by the number of heads (traffic grows with
+# kernel at H=4 (125.5 MB), scaled by the number of heads (traffic grows with
 # the heads processed). Valid only for the kernel source it was taken on.
-BWD_TRAFFIC = {"bytes": 4 * 124.686592e6,
-               "source_sha256": "45105d16dd5f6e9d5b2a0caa40252317694ff516b61b1b53c10eec4b1ce10159",
+BWD_TRAFFIC = {"bytes": 4 * 125.487616e6,
+               "source_sha256": "8350db18d4c24c3724c13a72d10f1deeb5185b7797efabc365b57967d687cc0b",
                "profile": "profiles/fa_bwd_kernel_b1h4_n16384_d128.md"}
 
 
