@@ -308,10 +308,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float s[128];
       {
         uint32_t sr[128];
-        tmem_ld32(tS + 0, sr + 0);
-        tmem_ld32(tS + 32, sr + 32);
-        tmem_ld32(tS + 64, sr + 64);
-        tmem_ld32(tS + 96, sr + 96);
+        tmem_ld64(tS + 0, sr + 0);
+        tmem_ld64(tS + 64, sr + 64);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
