@@ -451,6 +451,141 @@ def run_profile_case(args):
     return 0
 
 
+def run_next_rows(args):
+    """The widened rows on one GPU, one JSON line each (not part of the default
+    run): grouped K/V heads (H_kv = 4 and 1), a 4096-key sliding window, a
+    packed variable-length batch and the FP8 forward, all at d = 128 with 16
+    query heads and inputs larger than L2. Device-timed with CUDA events over
+    --steps calls after --warmup; TFLOP/s count only the visible (query, key)
+    pairs: 4 d per pair forward, 2.5 times that backward."""
+    import numpy as np
+    import torch
+
+    import exact_attention_118_b200 as fa
+
+    peak, _, _, peak_kind = _peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sp = torch.cuda.current_stream(dev).cuda_stream
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    d, H = 128, 16
+    scale = d ** -0.5
+
+    def rnd(*shape):
+        return torch.randn(*shape, device=dev, generator=g).to(torch.bfloat16)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        fa.check_device_error()
+        return a.elapsed_time(b) / args.steps
+
+    def check(st):
+        if st != fa.FA_OK:
+            raise RuntimeError(fa.fa_strerror(st))
+
+    def pairs(L, wl, wr):
+        i = np.arange(L)
+        lo = np.zeros(L) if wl < 0 else np.maximum(0, i - wl)
+        hi = np.full(L, L - 1) if wr < 0 else np.minimum(L - 1, i + wr)
+        return float(np.sum(hi - lo + 1))
+
+    def emit(row, config, ms_f, ms_b, vis_pairs, dtype="bf16", fwd_peak=None):
+        ff = 4.0 * d * H * vis_pairs
+        line = {"row": row, "metric": "attention TFLOPS/s of visible work", "unit": UNIT, "dtype": dtype,
+                "data": "synthetic", "config": config, "steps": args.steps, "warmup": args.warmup,
+                "fwd_ms": ms_f, "fwd_tflops": ff / ms_f / 1e9}
+        line["fwd_frac_of_peak"] = line["fwd_tflops"] / (fwd_peak or peak)
+        if ms_b is not None:
+            line.update({"bwd_ms": ms_b, "bwd_tflops": 2.5 * ff / ms_b / 1e9,
+                         "bwd_frac_of_peak": 2.5 * ff / ms_b / 1e9 / peak,
+                         "value": 3.5 * ff / (ms_f + ms_b) / 1e9})
+        else:
+            line["value"] = line["fwd_tflops"]
+        line["peak"] = fwd_peak or peak
+        line["peak_kind"] = peak_kind if fwd_peak is None else f"{peak_kind} bf16 x 2 (nominal e4m3:bf16 ratio)"
+        print(json.dumps(line), flush=True)
+
+    N = 16384
+    # Grouped K/V heads, causal.
+    for Hkv in (4, 1):
+        q, do = rnd(1, H, N, d), rnd(1, H, N, d)
+        k, v = rnd(1, Hkv, N, d), rnd(1, Hkv, N, d)
+        o = torch.empty_like(q)
+        lse = torch.empty(1, H, N, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        wsb = fa.fa_bwd_gqa_workspace_size(1, H, Hkv, N, d)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        fwd = lambda: check(fa.fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                          lse.data_ptr(), 1, H, Hkv, N, d, scale, 1, fa.FA_BF16, sp))
+        bwd = lambda: check(fa.fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                          lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                          dv.data_ptr(), ws.data_ptr(), wsb, 1, H, Hkv, N, d, scale, 1, sp))
+        fwd()
+        emit(f"gqa_hkv{Hkv}", {"workload": f"causal grouped-query attention, B=1 H={H} H_kv={Hkv} N={N} d={d}"},
+             timed(fwd), timed(bwd), pairs(N, -1, 0))
+    # Sliding window.
+    wl = 4095
+    q, k, v, do = rnd(1, H, N, d), rnd(1, H, N, d), rnd(1, H, N, d), rnd(1, H, N, d)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, H, N, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    wsb = fa.fa_bwd_gqa_workspace_size(1, H, H, N, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    fwd = lambda: check(fa.fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                         lse.data_ptr(), 1, H, H, N, d, scale, wl, 0, fa.FA_BF16, sp))
+    bwd = lambda: check(fa.fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                         lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                         ws.data_ptr(), wsb, 1, H, H, N, d, scale, wl, 0, sp))
+    fwd()
+    emit("window_4095_0", {"workload": f"sliding-window causal attention (4096 keys), B=1 H={H} N={N} d={d}"},
+         timed(fwd), timed(bwd), pairs(N, wl, 0))
+    # Packed variable length: 16 sequences of 512..8192 tokens (seeded), causal.
+    lens = [int(x) for x in np.random.default_rng(5).integers(512, 8193, 16)]
+    T = sum(lens)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev)
+    q, k, v, do = rnd(T, H, d), rnd(T, H, d), rnd(T, H, d), rnd(T, H, d)
+    o = torch.empty_like(q)
+    lse = torch.empty(H, T, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    wsb = fa.fa_bwd_varlen_workspace_size(len(lens), T, H, H, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    mx = max(lens)
+    fwd = lambda: check(fa.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                         lse.data_ptr(), cu.data_ptr(), len(lens), mx, T, H, H, d, scale, -1, 0,
+                                         fa.FA_BF16, sp))
+    bwd = lambda: check(fa.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),  # noqa: E731
+                                         lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                         cu.data_ptr(), ws.data_ptr(), wsb, len(lens), mx, T, H, H, d, scale, -1, 0,
+                                         sp))
+    fwd()
+    emit("varlen_16seq", {"workload": f"packed variable-length causal batch, 16 sequences of 512..8192 tokens "
+                                      f"(T={T}, longest {mx}), H={H} d={d}", "lengths": lens},
+         timed(fwd), timed(bwd), sum(pairs(L, -1, 0) for L in lens))
+    # FP8 forward.
+    for causal in (0, 1):
+        q8, k8, v8 = ((torch.randn(1, H, N, d, device=dev, generator=g) * 100).to(torch.float8_e4m3fn)
+                      .view(torch.uint8) for _ in range(3))
+        o = torch.empty(1, H, N, d, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(1, H, N, device=dev)
+        fwd = lambda: check(fa.fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), o.data_ptr(),  # noqa: E731
+                                          lse.data_ptr(), 1, H, H, N, d, scale, 0.01, 0.01, 0.01, -1,
+                                          0 if causal else -1, fa.FA_BF16, sp))
+        fwd()
+        emit(f"fp8_fwd{'_causal' if causal else ''}",
+             {"workload": f"FP8 (e4m3) forward{', causal' if causal else ''}, B=1 H={H} N={N} d={d}"},
+             timed(fwd), None, pairs(N, -1, 0 if causal else -1), dtype="e4m3", fwd_peak=2.0 * peak)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -461,7 +596,11 @@ def main():
     ap.add_argument("--profile-case", type=int, default=0, metavar="HEADS",
                     help="run untimed fwd+bwd launches with this many heads (for ncu) and exit")
     ap.add_argument("--causal", action="store_true", help="with --profile-case: causal mask")
+    ap.add_argument("--next-rows", action="store_true",
+                    help="time the widened rows (grouped K/V, window, variable length, FP8), one line each")
     args = ap.parse_args()
+    if args.next_rows:
+        return run_next_rows(args)
     if args.profile_case:
         return run_profile_case(args)
     if args.warmup < 3 and args.impl == "native":
