@@ -18,12 +18,16 @@
  *   Layout     q, k, v, o, dO, dq, dk, dv are dense, contiguous [B, H, N, d]
  *              row-major tensors (the [B, H, N, d] shape of the pasted
  *              pseudocode on the blog page, step 1). lse is [B, H, N] fp32.
+ *              The grouped-query, variable-length and FP8 calls below state
+ *              where theirs differ.
  *   dtypes     q, k, v, dO, dq, dk, dv: bf16. o: bf16 or fp32 in fa_fwd
  *              (o_dtype), bf16 in fa_bwd.
  *   Pointers   device pointers (CUDA global memory of the current device),
  *              each 16-byte aligned. The caller owns every buffer, including
- *              the backward workspace. The library allocates no device memory;
- *              it keeps only a small host-side cache of launch descriptors.
+ *              the backward workspace. The library allocates no device memory
+ *              at run time. Across calls it keeps only the per-device address
+ *              of fa_bwd_noalloc's fixed scratch array (part of the loaded
+ *              module) and, per host thread, the last CUDA error code.
  *   Sizes      B >= 1, H >= 1, N >= 1 (any value, ragged tails are handled),
  *              d in {64, 128}, B*H*N < 2^31.
  *   scale      the factor applied to Q K^T (1/sqrt(d) in the pages' pseudocode,
