@@ -47,7 +47,7 @@ WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then caus
 # kernel at H=4 (125.5 MB), scaled by the number of heads (traffic grows with
 # the heads processed). Valid only for the kernel source it was taken on.
 BWD_TRAFFIC = {"bytes": 4 * 125.487616e6,
-               "source_sha256": "fde83a89af27b80fb596966a03450f0611287a348ea081c8732eb12fadb4b12f",
+               "source_sha256": "f8e8736c39689d10022fb23129c48e19d8252ba7661ff6a4992b63a56b93268a",
                "profile": "profiles/fa_bwd_kernel_b1h4_n16384_d128.md"}
 
 

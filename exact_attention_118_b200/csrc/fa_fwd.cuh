@@ -353,27 +353,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t pk[64];
       if (FP8) {
         // Four e4m3 probabilities per TMEM column: P fills 32 columns.
+        const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
+        float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(fmaf(s[4 * c], lam, neg_m));
-          const float p1 = ex2(fmaf(s[4 * c + 1], lam, neg_m));
-          const float p2 = ex2(fmaf(s[4 * c + 2], lam, neg_m));
-          const float p3 = ex2(fmaf(s[4 * c + 3], lam, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          rs0 += p2;
-          rs1 += p3;
-          pk[c] = pack_e4m3x4(p0, p1, p2, p3);
+          const float2 x0 = ffma2(make_float2(s[4 * c], s[4 * c + 1]), lam2, negm2);
+          const float2 x1 = ffma2(make_float2(s[4 * c + 2], s[4 * c + 3]), lam2, negm2);
+          const float2 p01 = make_float2(ex2(x0.x), ex2(x0.y)), p23 = make_float2(ex2(x1.x), ex2(x1.y));
+          rs = fadd2(rs, p01);
+          rs = fadd2(rs, p23);
+          pk[c] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
         }
+        rs0 = rs.x;
+        rs1 = rs.y;
       } else {
+        const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
+        float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(fmaf(s[2 * c], lam, neg_m));
-          const float p1 = ex2(fmaf(s[2 * c + 1], lam, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          pk[c] = pack_bf16(p0, p1);
+          const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), lam2, negm2);
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          rs = fadd2(rs, pp);
+          pk[c] = pack_bf16(pp.x, pp.y);
         }
+        rs0 = rs.x;
+        rs1 = rs.y;
       }
       l = l * alpha + (rs0 + rs1);
       tmem_st32(tS + 0, pk + 0);
