@@ -215,6 +215,7 @@ struct BwdParams {
   int Hkv;        // K/V heads; query heads [g*H/Hkv, (g+1)*H/Hkv) share K/V head g
   int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv)
   int wl, wr;     // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
+  int sched_groups;  // causal launch order: number of unit groups (1 <= sched_groups <= BH)
   const int* cu_seqlens;  // packed variable length ([T, heads, D] tensors): [B + 1] prefix sums; else nullptr
   int T;                  // packed rows (variable length only); N is then the longest length
   int N;
@@ -297,11 +298,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Causal: key tile 0 sees every query tile, so low j first (heaviest).
+  // Causal: key tile 0 sees every query tile, so low j first (heaviest),
+  // within sched_groups groups of units, each small enough that its Q, dO and
+  // dQ accumulator stay in L2 (grouped_order). Otherwise unit-major.
   int j, unit;
   if (MASK == kMaskCausal) {
-    j = static_cast<int>(blockIdx.x) / p.BH;
-    unit = static_cast<int>(blockIdx.x) % p.BH;
+    grouped_order(static_cast<int>(blockIdx.x), p.BH, p.sched_groups, p.n_kv, j, unit);
   } else {
     unit = static_cast<int>(blockIdx.x) / p.n_kv;
     j = static_cast<int>(blockIdx.x) % p.n_kv;

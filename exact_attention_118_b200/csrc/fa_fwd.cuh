@@ -59,6 +59,7 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e) (FP8: times the Q and K dequantisation scales)
   float o_scale;     // multiplies O in the epilogue: 1, or the V dequantisation scale (FP8)
   int wl, wr;        // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
+  int sched_groups;  // causal launch order: number of head groups (1 <= sched_groups <= BH)
   const int* cu_seqlens;  // packed variable length: [B + 1] prefix sums of the lengths; else nullptr
   int T;                  // packed rows (variable length only); N is then the longest length
 };
@@ -112,12 +113,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Causal: heaviest query tiles first across all heads. Otherwise head-major
-  // so CTAs that read the same K/V run together and share it through L2.
+  // Causal: heads in sched_groups groups, each small enough that its K/V
+  // stays in L2 and large enough that its heaviest query tiles (started
+  // first) finish with the rest; see grouped_order. Otherwise head-major, so
+  // CTAs that read the same K/V run together.
   int pair, bh;
   if (MASK == kMaskCausal) {
-    pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / p.BH;
-    bh = static_cast<int>(blockIdx.x) % p.BH;
+    int t;
+    grouped_order(static_cast<int>(blockIdx.x), p.BH, p.sched_groups, p.n_pairs, t, bh);
+    pair = p.n_pairs - 1 - t;
   } else {
     bh = static_cast<int>(blockIdx.x) / p.n_pairs;
     pair = static_cast<int>(blockIdx.x) % p.n_pairs;

@@ -130,6 +130,35 @@ unsigned helper_grid(long long threads_needed) {
   return static_cast<unsigned>(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
 }
 
+// Causal grids launch the heaviest tiles first, which spreads the CTAs that
+// run at the same time over many heads. Splitting the heads (units) into
+// groups, heaviest-first within each, keeps a group's streamed operands in L2
+// (about 64 MB of its 126 MB). A group must also hold enough work that its
+// heaviest CTA (about 2 tiles' worth of steps per tile of the longest axis)
+// finishes no later than the group's other CTAs: with `tiles` tiles per unit
+// and work ~ tiles^2 per unit spread over the SMs, that needs a group of at
+// least 2 * SMs / tiles units. Working sets up to twice the L2 gain nothing
+// from grouping (measured), so they keep one group: the global
+// heaviest-first order. Returns the number of groups.
+int sched_groups(long long bytes_per_unit, int units, int tiles) {
+  if (bytes_per_unit * units <= (256ll << 20)) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+    sms = 148;
+  const long long budget = 64ll << 20;
+  long long g_max = bytes_per_unit > 0 ? budget / bytes_per_unit : units;
+  if (g_max < 1) g_max = 1;
+  long long g_min = tiles > 0 ? (2ll * sms + tiles - 1) / tiles : 1;
+  if (g_min < 1) g_min = 1;
+  long long groups = (units + g_max - 1) / g_max;  // fit in L2
+  const long long most = units / g_min;            // no group below g_min
+  if (groups > most) groups = most;
+  if (groups < 1) groups = 1;
+  if (groups > units) groups = units;
+  return static_cast<int>(groups);
+}
+
 // The mask a call asks for, reduced to one of the kernels' three modes. A
 // window wider than the sequence on a side is no bound on that side, so a
 // band that bounds nothing is the unmasked kernel and a band bounded only on
@@ -287,6 +316,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.n_split = n_split;
   p.wl = mask.wl;
   p.wr = mask.wr;
+  // Per unit: Q and dO (bf16) and the fp32 dQ accumulator of its query heads.
+  p.sched_groups = sched_groups(static_cast<long long>(g.H / g.Hkv / n_split) * g.N * D * 8, p.BH, (g.N + 127) / 128);
   p.cu_seqlens = g.cu;
   p.T = g.T;
   p.N = g.N;
@@ -376,6 +407,7 @@ fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, v
   p.n_pairs = (g.N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_scale = 1.f;
+  p.sched_groups = sched_groups(2ll * g.N * d * 2, g.B * g.H, p.n_pairs);  // K and V of a head, bf16
   const Mask m = resolve_mask(window_left, window_right, g.N);
   p.wl = m.wl;
   p.wr = m.wr;
@@ -410,6 +442,7 @@ fa_status fwd_fp8_impl(const Geom& g, const void* q8, const void* k8, const void
   p.n_pairs = (g.N + 255) / 256;
   p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
   p.o_scale = v_scale;
+  p.sched_groups = sched_groups(2ll * g.N * 128, g.B * g.H, p.n_pairs);  // K and V of a head, e4m3
   const Mask m = resolve_mask(window_left, window_right, g.N);
   p.wl = m.wl;
   p.wr = m.wr;

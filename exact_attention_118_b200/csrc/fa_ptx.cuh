@@ -397,6 +397,31 @@ __device__ __forceinline__ void seq_range(const int* cu, int b, int T, int max_l
   L = min(min(max(e, s0), T) - s0, max_len);
 }
 
+// Causal launch order. The units (heads) are split into `groups` groups of
+// near-equal size, the first BH % groups one unit larger; within a group,
+// tile t of every unit comes before tile t + 1 (the caller orders tiles
+// heaviest first). Maps block b to (tile, unit); a bijection onto
+// [0, n_tiles) x [0, BH) for 1 <= groups <= BH.
+__device__ __forceinline__ void grouped_order(int b, int BH, int groups, int n_tiles, int& tile, int& unit) {
+  const int base = BH / groups, extra = BH % groups;
+  const int big = (base + 1) * n_tiles;
+  int r, gc, u0;
+  if (b < extra * big) {
+    const int gi = b / big;
+    r = b - gi * big;
+    gc = base + 1;
+    u0 = gi * (base + 1);
+  } else {
+    const int b2 = b - extra * big, small = base * n_tiles;
+    const int gi = b2 / small;
+    r = b2 - gi * small;
+    gc = base;
+    u0 = extra * (base + 1) + gi * base;
+  }
+  tile = r / gc;
+  unit = u0 + r % gc;
+}
+
 // Attention masks the kernels are instantiated for. Band: key j is visible
 // to query i iff i - wl <= j <= i + wr (the local window), wl, wr >= 0.
 enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskBand = 2 };
