@@ -44,10 +44,10 @@ WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then caus
 
 # DRAM traffic of one non-causal main backward launch of the workload above:
 # dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the same
-# kernel at H=4 (125.5 MB), scaled by the number of heads (traffic grows with
+# kernel at H=4 (124.3 MB), scaled by the number of heads (traffic grows with
 # the heads processed). Valid only for the kernel source it was taken on.
-BWD_TRAFFIC = {"bytes": 4 * 125.487616e6,
-               "source_sha256": "f8e8736c39689d10022fb23129c48e19d8252ba7661ff6a4992b63a56b93268a",
+BWD_TRAFFIC = {"bytes": 4 * 124.274432e6,
+               "source_sha256": "869879acb85a01665f6f8056b06b06f557cee23241e34711e08c002076478fa9",
                "profile": "profiles/fa_bwd_kernel_b1h4_n16384_d128.md"}
 
 
