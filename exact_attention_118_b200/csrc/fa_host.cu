@@ -56,6 +56,8 @@ fa_status check_sizes(int B, int H, int N, int d, float scale, int causal) {
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+  // Tile and band bounds are formed in 32-bit ints (up to about 2 N).
+  if (N > (1 << 29)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }

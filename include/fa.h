@@ -29,7 +29,7 @@
  *              of fa_bwd_noalloc's fixed scratch array (part of the loaded
  *              module) and, per host thread, the last CUDA error code.
  *   Sizes      B >= 1, H >= 1, N >= 1 (any value, ragged tails are handled),
- *              d in {64, 128}, B*H*N < 2^31.
+ *              d in {64, 128}, B*H*N < 2^31, N <= 2^29 (T <= 2^29 packed).
  *   scale      the factor applied to Q K^T (1/sqrt(d) in the pages' pseudocode,
  *              step 3); any finite value > 0.
  *   causal     0: every key visible. 1: key j visible to query i iff j <= i

@@ -207,3 +207,10 @@ def test_fp8_forward_rejects_bad_arguments():
     assert call(vs=float("inf")) == fa.FA_ERR_INVALID_ARG
     assert call(vs=float("nan")) == fa.FA_ERR_INVALID_ARG
     assert call(Hkv=3) == fa.FA_ERR_INVALID_ARG
+
+
+def test_sequence_length_limit():
+    # N up to 2^29 keeps the kernels' 32-bit tile and band arithmetic exact.
+    assert fa.fa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, (1 << 29) + 1, 64, 0.1, 0, fa.FA_BF16,
+                     None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_workspace_size(1, 1, (1 << 29) + 1, 64) == 0
