@@ -42,13 +42,16 @@ B, H, N, D = 1, 16, 16384, 128
 SEED = 3
 WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then causal"
 
-# DRAM traffic of one non-causal main backward launch of the workload above:
-# dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of the same
-# kernel at H=4 (124.3 MB), scaled by the number of heads (traffic grows with
-# the heads processed). Valid only for the kernel source it was taken on.
-BWD_TRAFFIC = {"bytes": 4 * 124.274432e6,
-               "source_sha256": "869879acb85a01665f6f8056b06b06f557cee23241e34711e08c002076478fa9",
-               "profile": "profiles/fa_bwd_kernel_b1h4_n16384_d128.md"}
+# DRAM traffic of one non-causal main backward launch of the workload above
+# (B=1, H=16, N=16384, d=128): dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture of that very launch shape. None until a capture of the
+# current kernel source exists; a number taken on other source is not used.
+BWD_TRAFFIC = {"bytes": None, "read": None, "write": None,
+               "shape": "B=1 H=16 N=16384 d=128, non-causal, one launch",
+               "source_sha256": None}
+# Dense bf16 tensor-core peak of a B200 as the vendor states it, reported next
+# to the fraction of the measured peak.
+SPEC_BF16_TFLOPS = 2250.0
 
 
 def _flops(causal: bool):
@@ -359,9 +362,11 @@ def run_native(args):
     for c, tag in ((False, "noncausal"), (True, "causal")):
         ff, fb = _flops(c)
         passes[f"fwd_{tag}"] = {"ms": fwd_ms[c], "tflops": ff / fwd_ms[c] / 1e9,
-                                "frac_of_peak": ff / fwd_ms[c] / 1e9 / peak}
+                                "frac_of_peak": ff / fwd_ms[c] / 1e9 / peak,
+                                "frac_of_spec": ff / fwd_ms[c] / 1e9 / SPEC_BF16_TFLOPS}
         passes[f"bwd_{tag}"] = {"ms": per[c]["bwd_ms"], "tflops": fb / per[c]["bwd_ms"] / 1e9,
                                 "frac_of_peak": fb / per[c]["bwd_ms"] / 1e9 / peak,
+                                "frac_of_spec": fb / per[c]["bwd_ms"] / 1e9 / SPEC_BF16_TFLOPS,
                                 "main_kernel_ms": per[c]["bwd_main_ms"]}
 
     # Roofline of the dominant kernel: the main backward kernel, non-causal
@@ -371,12 +376,19 @@ def run_native(args):
     traffic = None
     if BWD_TRAFFIC["bytes"] is not None and BWD_TRAFFIC["source_sha256"] == _bwd_source_sha():
         traffic = BWD_TRAFFIC["bytes"]
+    # Algorithmic bytes of one launch: Q, K, V, dO read and dK, dV written in
+    # bf16, lse2 and D read, and the fp32 dQ accumulator written once.
+    alg_bytes = B * H * N * (6 * D * 2 + 2 * 4 + D * 4)
     roofline = {"kernel": "fa_bwd_kernel<128, non-causal> (main backward)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": traffic, "traffic_source": BWD_TRAFFIC["profile"] if traffic else None,
-                "algorithmic_flops_per_launch": bwd_nc, "avg_launch_ms": main_ms,
+                "traffic": traffic,
+                "traffic_shape": BWD_TRAFFIC["shape"] if traffic else None,
+                "traffic_over_algorithmic_bytes": traffic / alg_bytes if traffic else None,
+                "algorithmic_flops_per_launch": bwd_nc, "algorithmic_bytes_per_launch": alg_bytes,
+                "avg_launch_ms": main_ms,
                 "peak_kind": f"{peak_kind} bf16 dense (burst); sustained {peak_sus}",
-                "frac_of_sustained": achieved / peak_sus}
+                "frac_of_sustained": achieved / peak_sus,
+                "frac_of_spec": achieved / SPEC_BF16_TFLOPS}
 
     # ---------------------------------------------------- end-to-end (host buffers)
     # A pipelined application loop: each step uploads its inputs from pinned
@@ -459,6 +471,8 @@ def run_native(args):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (Q,K,V,dO 67 MB each; 1.1 GB working set per step)"},
         "frac_of_peak": value / peak,
+        "frac_of_spec": value / SPEC_BF16_TFLOPS,
+        "peak": {"bf16_tflops": peak, "kind": peak_kind, "spec_bf16_tflops": SPEC_BF16_TFLOPS},
         "passes": passes,
         "roofline": roofline,
         "cpu_baseline": cpu_baseline,

@@ -24,6 +24,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa.h")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_BF16, FA_F32 = 0, 1
+FA_DEVERR_TIMEOUT, FA_DEVERR_SMEM_ALIGN, FA_DEVERR_SEQLENS = 1, 2, 4
 FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _P = ctypes.c_void_p
@@ -47,9 +48,11 @@ _SIGNATURES = {
     "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_get_device_error": (_I, [_P]),
+    "fa_decode_device_error": (_I, [ctypes.c_uint]),
     "fa_set_bwd_main_events": (_I, [_P, _P]),
     "fa_last_cuda_error": (_I, []),
     "fa_selftest_wait_timeout": (_I, [_P]),
+    "fa_selftest_exp2_fma": (_I, [_P, _P, ctypes.c_longlong, _P]),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -155,6 +158,10 @@ def fa_get_device_error(stream) -> int:
     return _lib.fa_get_device_error(stream)
 
 
+def fa_decode_device_error(word) -> int:
+    return _lib.fa_decode_device_error(word)
+
+
 def fa_set_bwd_main_events(before, after) -> int:
     return _lib.fa_set_bwd_main_events(before, after)
 
@@ -165,6 +172,10 @@ def fa_last_cuda_error() -> int:
 
 def fa_selftest_wait_timeout(stream) -> int:
     return _lib.fa_selftest_wait_timeout(stream)
+
+
+def fa_selftest_exp2_fma(x, y, n, stream) -> int:
+    return _lib.fa_selftest_exp2_fma(x, y, n, stream)
 
 
 def fa_strerror(status: int) -> str:

@@ -11,27 +11,25 @@
 //   dQ = scale * dS K,           dK = scale * dS^T Q.
 //
 // Main kernel: one CTA per (batch*K/V head, 128-key tile j); it loops over
-// 64-query tiles i (causal: only i with a visible query, the masked upper
-// triangle is skipped) of every query head reading that K/V head, and keeps
-// dK_j, dV_j accumulating in TMEM. Everything is
-// computed transposed (keys on TMEM lanes) so P^T and dS^T can feed the dV/dK
-// MMAs straight from TMEM:
-//   S^T  = K_j Q_i^T        (SS, M=128 keys, N=64 queries)   -> TMEM S[b]
-//   dP^T = V_j dO_i^T       (SS)                             -> TMEM dP[b]
+// 128-query tiles i (causal: only i >= j, the masked upper triangle is
+// skipped) of every query head reading that K/V head, and keeps dK_j, dV_j
+// accumulating in TMEM. Everything is computed transposed (keys on TMEM
+// lanes) so P^T and dS^T can feed the dV/dK MMAs straight from TMEM:
+//   S^T  = K_j Q_i^T        (SS, M=128 keys, N=128 queries)  -> TMEM
+//   dP^T = V_j dO_i^T       (SS)                             -> TMEM
 //   P^T  = 2^(lambda*S^T - lse2),  dS^T = scale * P^T * (dP^T - D)   (registers)
 //   dV  += P^T dO_i         (TS: A = P^T bf16 in TMEM)
 //   dK  += dS^T Q_i         (TS: A = dS^T bf16 in TMEM)
 //   dQ_i^T = K_j^T dS^T     (SS: A = K_j read MN-major, B = dS from smem)
 //   dQ_i^T is drained from TMEM by a warpgroup that stages it in shared
 //   memory and adds it into the fp32 dQ accumulator with TMA reduce-adds.
-// S and dP are double-buffered (b = iteration & 1) so the tensor core computes
-// tile i+1 while an elementwise warpgroup works on tile i; each buffer has its
-// own elementwise warpgroup, so the two groups overlap each other's waits.
+// All five products are N = 128 (or N = D) instructions; the TMEM regions are
+// single-buffered and their reuse is ordered as described at the kernel.
 //
-// Roles (512 threads): warp 0 TMA producer (Q, dO, lse2 and D tiles), warps 1
-// to 3 MMA issuers, warps 4-7 the dQ drain warpgroup (thread = head-dim row of
-// dQ^T), warps 8-11 and 12-15 two elementwise warpgroups (thread = key row)
-// that take alternate query tiles.
+// Roles (512 threads): warp 0 TMA producer (Q with its lse2 and D rows, dO),
+// warps 1 to 3 MMA issuers, warps 4-7 the dQ drain warpgroup (thread =
+// head-dim row of dQ^T), warps 8-11 and 12-15 two elementwise warpgroups
+// (thread = key row) that take query columns 0-63 and 64-127 of every tile.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -94,10 +92,16 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int part = static_cast<int>(tid % TPR);
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x / TPR;
-  for (long long row = tid / TPR; row < rows; row += stride) {
-    const size_t off = static_cast<size_t>(row) * D + part * 8;
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
-    const uint4 g = __ldg(reinterpret_cast<const uint4*>(dO + off));
+  // A warp covers 32 / TPR consecutive rows and steps through them together,
+  // so every lane runs the same iterations (the shuffles need the full warp);
+  // lanes whose row is past the end take part with zeros and store nothing.
+  const int lane = threadIdx.x & 31;
+  for (long long row0 = (tid - lane) / TPR; row0 < rows; row0 += stride) {
+    const long long row = row0 + lane / TPR;
+    const bool live = row < rows;
+    const size_t off = static_cast<size_t>(live ? row : 0) * D + part * 8;
+    const uint4 a = live ? __ldg(reinterpret_cast<const uint4*>(o + off)) : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 g = live ? __ldg(reinterpret_cast<const uint4*>(dO + off)) : make_uint4(0u, 0u, 0u, 0u);
     const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
     float s = 0.f;
@@ -110,6 +114,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_kernel(const __nv_bfloat16* __
     }
 #pragma unroll
     for (int w = TPR / 2; w >= 1; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
+    if (!live) continue;
     if (part == 0) {
       const long long bh = row / N, qi = row - bh * N;
       const size_t so = static_cast<size_t>(bh) * Np + qi;
@@ -140,17 +145,21 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_varlen_kernel(
   const int tid = static_cast<int>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int part = tid % TPR;
   const int stride = static_cast<int>(gridDim.x) * blockDim.x / TPR;
+  const int lane = threadIdx.x & 31;
   for (int b = blockIdx.y; b < B; b += gridDim.y) {
     int s0, L;
     seq_range(cu, b, T, max_len, s0, L);
     const int P = varlen_stat_start(s0, b);
     const int P_end = (b == B - 1) ? Sp : varlen_stat_start(s0 + L, b + 1);
     const int rows = L * H;
-    for (int r = tid / TPR; r < rows; r += stride) {
-      const int i = r / H, h = r - i * H;
+    // Warp-uniform row loop, as in fa_bwd_dot_kernel.
+    for (int r0 = (tid - lane) / TPR; r0 < rows; r0 += stride) {
+      const int r = r0 + lane / TPR;
+      const bool live = r < rows;
+      const int i = (live ? r : 0) / H, h = (live ? r : 0) - i * H;
       const size_t off = (static_cast<size_t>(s0 + i) * H + h) * D + part * 8;
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
-      const uint4 g = __ldg(reinterpret_cast<const uint4*>(dO + off));
+      const uint4 a = live ? __ldg(reinterpret_cast<const uint4*>(o + off)) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 g = live ? __ldg(reinterpret_cast<const uint4*>(dO + off)) : make_uint4(0u, 0u, 0u, 0u);
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
       const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
       float sum = 0.f;
@@ -163,6 +172,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dot_varlen_kernel(
       }
 #pragma unroll
       for (int w = TPR / 2; w >= 1; w >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, w);
+      if (!live) continue;
       if (part == 0) {
         const size_t so = static_cast<size_t>(h) * Sp + P + i;
         dsum[so] = sum;
@@ -206,14 +216,10 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
 
 // ------------------------------------------------------------------ main kernel
 struct BwdParams {
-  void* dk;       // bf16 [B, Hkv, N, D]      (n_split == 1)
-  void* dv;       // bf16 [B, Hkv, N, D]      (n_split == 1)
-  float* dk_acc;  // fp32 [B, Hkv, N, D], zeroed (n_split > 1)
-  float* dv_acc;  // fp32 [B, Hkv, N, D], zeroed (n_split > 1)
   int BH;         // batch * K/V heads * n_split: one CTA per (unit, 128-key tile)
   int H;          // query heads
   int Hkv;        // K/V heads; query heads [g*H/Hkv, (g+1)*H/Hkv) share K/V head g
-  int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv)
+  int n_split;    // CTAs that share one K/V head's query heads (divides H/Hkv); > 1: dK, dV add into fp32
   int wl, wr;     // band mask only: key j visible to query i iff i - wl <= j <= i + wr (0 <= wl, wr <= N)
   int sched_groups;  // causal launch order: number of unit groups (1 <= sched_groups <= BH)
   const int* cu_seqlens;  // packed variable length ([T, heads, D] tensors): [B + 1] prefix sums; else nullptr
@@ -222,78 +228,110 @@ struct BwdParams {
   int n_kv;          // ceil(N / 128)
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
+  // Rows of a ragged last key tile that the TMA store cannot clip (packed
+  // layout) are written by the threads themselves, here:
+  void* dk;          // bf16 [.., D] (n_split == 1)
+  void* dv;
+  float* dk_acc;     // fp32 [.., D], zeroed (n_split > 1)
+  float* dv_acc;
 };
 
+// Shared memory of the main kernel (bytes). A tile is 128 rows x D bf16, kept
+// as D/64 column chunks of [128 rows][128 B] with the 128-byte swizzle.
 template <int D>
 struct BwdLayout {
-  static constexpr int kKV = 128 * D * 2;  // K or V tile: 128 keys
-  static constexpr int kQT = 64 * D * 2;   // Q or dO tile: 64 queries
-  static constexpr int kStages = (D == 128) ? 3 : 4;  // Q/dO/lse2/D ring depth
-  static constexpr int kDSTile = 128 * 64 * 2;
+  static constexpr int kChunk = 128 * 128;              // one 64-column chunk of a 128-row tile
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kQS = (D == 128) ? 2 : 3;        // Q (+ lse2, D statistics) ring
+  static constexpr int kDOS = (D == 128) ? 1 : 2;       // dO ring
   static constexpr int kK = 0;
-  static constexpr int kV = kKV;
-  static constexpr int kQ = 2 * kKV;
-  static constexpr int kDO = kQ + kStages * kQT;
-  // [2] dS tiles [128 keys][64 queries].
-  static constexpr int kDS = kDO + kStages * kQT;
-  static constexpr int kStat = kDS + 2 * kDSTile;  // [kStages] x {lse2[64], D[64]}
-  // [2] fp32 staging halves for dQ_i (32 queries x D each), so one half is
-  // written while the TMA engine still reads the other.
+  static constexpr int kV = kTile;
+  static constexpr int kQ = 2 * kTile;
+  static constexpr int kDO = kQ + kQS * kTile;
+  // dS tile as the MN-major operand of dQ^T: [2 query groups of 64][128 keys][128 B].
+  static constexpr int kDS = kDO + kDOS * kTile;
+  static constexpr int kDSTile = 128 * 128 * 2;
+  // Two fp32 staging buffers for dQ^T, 32 queries x D each: one is written
+  // while the TMA engine still reads the other.
   static constexpr int kStgHalf = 32 * D * 4;
-  static constexpr int kStg = (kStat + kStages * 512 + 1023) & ~1023;
-  static constexpr int kBar = kStg + 2 * kStgHalf;
+  static constexpr int kStg = kDS + kDSTile;
+  static constexpr int kStat = kStg + 2 * kStgHalf;     // [kQS] x {lse2[128], D[128]} fp32
+  static constexpr int kBar = kStat + kQS * 1024;
   static constexpr int kBytes = kBar + 256;
   // The kernel checks that the dynamic shared memory base is 1 KB aligned
   // (it is: the window starts on a 1 KB boundary) instead of reserving slack.
   static constexpr int kAlloc = kBytes;
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+  // Epilogue staging of dK/dV, one slot per elementwise warp (8), from offset
+  // 0: K, V and the Q ring are free by then.
+  static constexpr int kEpiBf16 = 32 * D * 2;
+  static constexpr int kEpiF32 = 32 * D * 4;
+  static_assert(8 * kEpiF32 <= kDO, "epilogue staging must fit in K, V and the Q ring");
 };
 
 // Roles, one warpgroup each: warps 0-3 control (warp 0 TMA producer, warps 1-3
-// MMA issuers, warp 1 also TMEM owner), 4-7 dQ drain, 8-11 elementwise
-// (even iterations, TMEM buffer 0), 12-15 elementwise (odd iterations, buffer
-// 1). Launched at 128 registers per thread (512 x 128 = the 64K register
-// file; each SM sub-partition holds one warp of every warpgroup); the groups
-// then move to 56 / 104 / 176 / 176, which sums to the same 512 per slot.
+// MMA issuers X, Y, Z; warp 1 also owns TMEM), 4-7 dQ drain, 8-11 and 12-15
+// elementwise (query columns 0-63 and 64-127 of every tile). Launched at 128
+// registers per thread (512 x 128 = the 64K register file; each SM
+// sub-partition holds one warp of every warpgroup); the groups then move to
+// 56 / 152 / 152 / 152, which sums to the same 512 per slot.
 constexpr int kBwdThreads = 512;
-constexpr int kRegCtl = 56, kRegDrain = 104, kRegElem = 176;
+constexpr int kRegCtl = 56, kRegDrain = 152, kRegElem = 152;
 static_assert(kRegCtl + kRegDrain + 2 * kRegElem == 512, "register split must equal the launch budget");
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Main backward kernel: one CTA per (batch*K/V head*share, 128-key tile j),
+// iterating over the 128-query tiles that see a key of the tile.
+//
+// TMEM (512 columns): S^T [0,128) with P^T (bf16) written over it, dP^T
+// [128,256) with dS^T (bf16) written over it and then dQ^T over both, dV at
+// 256, dK at 256 + D. Every region is single-buffered; reuse is ordered
+// either by one issuing thread (tcgen05.mma from one thread execute in issue
+// order) or by a barrier:
+//   X: dV(i) [after P^T(i)], then S^T(i+1) over S^T/P^T(i).
+//   Y: dK(i) [after dS^T(i)], then dQ^T(i) over dP^T/dS^T(i).
+//   Z: dP^T(i+1) over dQ^T(i), after the drain has copied dQ^T(i) out.
+// The elementwise groups turn S^T(i) into P^T(i) while Y and Z work on
+// iteration i-1's dK, dQ^T and the next dP^T, and turn dP^T(i) into dS^T(i)
+// while X computes dV(i) and S^T(i+1).
 template <int D, int MASK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_lse2,
-                  const __grid_constant__ CUtensorMap tm_dsum, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dsum, const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using L = BwdLayout<D>;
-  constexpr int QS = L::kStages;
+  constexpr int QS = L::kQS;
+  constexpr int DOS = L::kDOS;
   constexpr int KCH = D / 64;
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0u) {  // uniform over the CTA: nothing started yet
-    if (threadIdx.x == 0) atomicOr(&g_device_error, FA_DEVERR_SMEM_ALIGN);
+    if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrSmemAlign);
     return;
   }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars;
-  uint64_t* qd_full = kv_full + 1;      // [QS]
-  uint64_t* qd_empty = qd_full + QS;    // [QS]
-  uint64_t* s_full = qd_empty + QS;     // [2]
-  uint64_t* dp_full = s_full + 2;       // [2]
-  uint64_t* p_full = dp_full + 2;       // [2]
-  uint64_t* ds_full = p_full + 2;       // [2]
-  uint64_t* dq_full = ds_full + 2;      // [2]
-  uint64_t* dq_empty = dq_full + 2;     // [2]
-  uint64_t* y_done = dq_empty + 2;      // [2] dK of the buffer's last iteration done
-  uint64_t* acc_full = y_done + 2;
+  uint64_t* q_full = kv_full + 1;       // [QS] Q tile + statistics landed
+  uint64_t* q_empty = q_full + QS;      // [QS] S^T (X) and dK (Y) done reading
+  uint64_t* do_full = q_empty + QS;     // [DOS]
+  uint64_t* do_empty = do_full + DOS;   // [DOS] dP^T (Z) and dV (X) done reading
+  uint64_t* s_full = do_empty + DOS;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* dp_full = p_full + 1;
+  uint64_t* ds_full = dp_full + 1;
+  uint64_t* dq_full = ds_full + 1;
+  uint64_t* dq_empty = dq_full + 1;
+  uint64_t* acc_full = dq_empty + 1;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((1 + 2 * QS + 2 * DOS + 8) * 8 + 8 <= 256, "barrier region");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -324,37 +362,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int stat0 = packed ? varlen_stat_start(s0, bkv / p.Hkv) : 0;
   const int group = p.H / p.Hkv / p.n_split;   // query heads of this CTA
   const int qh0 = (packed ? 0 : (bkv / p.Hkv) * p.H) + (bkv % p.Hkv) * (p.H / p.Hkv) + (unit % p.n_split) * group;
-  const int n_q = (N + 63) / 64;
-  // 64-query tiles [i_start, i_end) that see a key of this tile; never empty,
-  // since key 128*j < N sees itself.
+  const int n_q = (N + 127) / 128;
+  // 128-query tiles [i_start, i_end) that see a key of this tile; never
+  // empty, since key 128*j < N sees itself.
   int i_start = 0, i_end = n_q;
-  if (MASK == kMaskCausal) i_start = 2 * j;
+  if (MASK == kMaskCausal) i_start = j;
   if (MASK == kMaskBand) {
-    i_start = max(0, j * 128 - p.wr) / 64;
-    i_end = min(n_q, min(j * 128 + 127 + p.wl, N - 1) / 64 + 1);
+    i_start = max(0, j * 128 - p.wr) / 128;
+    i_end = min(n_q, min(j * 128 + 127 + p.wl, N - 1) / 128 + 1);
   }
   const int n_iq = i_end - i_start;  // query tiles per head
   const int n_it = group * n_iq;
-  auto q_start = [&](int it) { return (i_start + it % n_iq) * 64; };
+  auto q_start = [&](int it) { return (i_start + it % n_iq) * 128; };
   auto q_head = [&](int it) { return qh0 + it / n_iq; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < QS; ++s) {
-      mbar_init(qd_full + s, 1);
-      mbar_init(qd_empty + s, 2);  // one release per MMA issuer
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 2);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(dp_full + b, 1);
-      mbar_init(p_full + b, 4);   // one arrival per warp of the elementwise group
-      mbar_init(ds_full + b, 4);
-      mbar_init(dq_full + b, 1);
-      mbar_init(dq_empty + b, 4);
-      mbar_init(y_done + b, 1);
+    for (int s = 0; s < DOS; ++s) {
+      mbar_init(do_full + s, 1);
+      mbar_init(do_empty + s, 2);
     }
-    mbar_init(acc_full, 2);   // last dV (X) and last dK (Y)
-    mbar_init(mma_done, 3);   // one per MMA issuer
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 8);    // one arrival per elementwise warp
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 8);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 4);  // one arrival per drain warp
+    mbar_init(acc_full, 2);  // last dV (X) and last dK + dQ^T (Y)
+    mbar_init(mma_done, 3);  // one per MMA issuer
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -364,13 +403,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int wg = warp >> 2;
-  // TMEM columns: S[b] at 64*b, dP[b] at 128 + 64*b, dV at 256, dK at 256 + D.
-  const uint32_t t_dv = 256, t_dk = 256 + D;
-  constexpr uint32_t kStageTx = 2 * L::kQT + 512;
+  constexpr uint32_t t_dp = 128, t_dv = 256, t_dk = 256 + D;
+  constexpr uint32_t kQTx = L::kTile + 1024;  // Q tile + lse2[128] + D[128]
 
   if (wg == 0) setmaxnreg_dec<kRegCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Loads in the order they are needed: Q(i) (needed by S^T(i)), then
+    // dO(i) (needed by dP^T(i), which comes later).
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
@@ -379,129 +419,137 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_dq);
       prefetch_tmap(&tm_lse2);
       prefetch_tmap(&tm_dsum);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
       for (int c = 0; c < KCH; ++c) {
-        tma_load_3d(smem + L::kK + c * 16384, &tm_k, kv_full, c * 64, s0 + j * 128, kvh);
-        tma_load_3d(smem + L::kV + c * 16384, &tm_v, kv_full, c * 64, s0 + j * 128, kvh);
+        tma_load_3d(smem + L::kK + c * L::kChunk, &tm_k, kv_full, c * 64, s0 + j * 128, kvh);
+        tma_load_3d(smem + L::kV + c * L::kChunk, &tm_v, kv_full, c * 64, s0 + j * 128, kvh);
       }
-      int issued = 0;
+      int q_issued = 0, do_issued = 0;
       for (int it = 0; it < n_it; ++it) {
-        const int s = it % QS, u = it / QS;
-        if (it >= QS && !wait_parity(qd_empty + s, (u - 1) & 1, abort_flag)) break;
         const int q0 = q_start(it), bhq = q_head(it);
-        uint8_t* st = smem + L::kStat + s * 512;
-        mbar_arrive_expect_tx(qd_full + s, kStageTx);
-        for (int c = 0; c < KCH; ++c) {
-          tma_load_3d(smem + L::kQ + s * L::kQT + c * 8192, &tm_q, qd_full + s, c * 64, s0 + q0, bhq);
-          tma_load_3d(smem + L::kDO + s * L::kQT + c * 8192, &tm_do, qd_full + s, c * 64, s0 + q0, bhq);
-        }
-        tma_load_2d(st, &tm_lse2, qd_full + s, stat0 + q0, bhq);
-        tma_load_2d(st + 256, &tm_dsum, qd_full + s, stat0 + q0, bhq);
-        issued = it + 1;
+        const int s = it % QS;
+        if (it >= QS && !wait_parity(q_empty + s, (it / QS - 1) & 1, abort_flag)) break;
+        uint8_t* st = smem + L::kStat + s * 1024;
+        mbar_arrive_expect_tx(q_full + s, kQTx);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(smem + L::kQ + s * L::kTile + c * L::kChunk, &tm_q, q_full + s, c * 64, s0 + q0, bhq);
+        tma_load_2d(st, &tm_lse2, q_full + s, stat0 + q0, bhq);
+        tma_load_2d(st + 512, &tm_dsum, q_full + s, stat0 + q0, bhq);
+        q_issued = it + 1;
+        const int t = it % DOS;
+        if (it >= DOS && !wait_parity(do_empty + t, (it / DOS - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(do_full + t, L::kTile);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(smem + L::kDO + t * L::kTile + c * L::kChunk, &tm_do, do_full + t, c * 64, s0 + q0, bhq);
+        do_issued = it + 1;
       }
+      // Every copy this thread started must land before the CTA exits.
       wait_parity_drain(kv_full, 0);
-      for (int it = max(0, issued - QS); it < issued; ++it) wait_parity_drain(qd_full + it % QS, (it / QS) & 1);
+      for (int it = max(0, q_issued - QS); it < q_issued; ++it) wait_parity_drain(q_full + it % QS, (it / QS) & 1);
+      for (int it = max(0, do_issued - DOS); it < do_issued; ++it)
+        wait_parity_drain(do_full + it % DOS, (it / DOS) & 1);
     }
   } else if (warp >= 1 && warp <= 3) {
     // ------------------------------------------------------- MMA issuers
-    // Issuing one tcgen05.mma costs the issuing thread about 100 cycles
-    // (measured), longer than a 128 x 64 x 16 product takes on the tensor
-    // core, so three threads share the 32 instructions of an iteration:
-    // X (warp 1) issues S^T and dV, Y (warp 2) dP^T and dK, Z (warp 3) dQ^T.
-    // X and Y meet at TMEM buffer S[b]: S^T(it+2) may overwrite it only after
-    // dK(it) has read dS^T from it (barrier y_done[b]; dV(it) is X's own and
-    // runs first). X and Y read the Q/dO stage, so qd_empty takes one release
-    // from each.
+    // Three threads share the 40 instructions of an iteration, so that
+    // products that do not depend on each other are in the tensor pipe
+    // together: X (warp 1) dV and S^T, Y (warp 2) dK and dQ^T, Z (warp 3) dP^T.
     if (lane == 0) {
-      const bool is_x = (warp == 1), is_z = (warp == 3);
-      constexpr uint32_t kIdST = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T: K-major A and B
-      constexpr uint32_t kIdAcc = idesc_bf16(128, D, 0, 1);  // dV, dK: A TMEM, B MN-major
-      constexpr uint32_t kIdDQ = idesc_bf16(D, 64, 1, 1);    // dQ^T: A, B MN-major
+      constexpr uint32_t kIdST = idesc_bf16(128, 128, 0, 0);  // S^T, dP^T: K-major A and B
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, 0, 1);   // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t kIdDQ = idesc_bf16(D, 128, 1, 1);    // dQ^T: A, B MN-major
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t do_addr = smem_u32(smem + L::kDO);
       const uint32_t ds_addr = smem_u32(smem + L::kDS);
 
-      // X^T = A_j Y^T, A_j a 128-row K/V tile, Y a 64-row Q/dO tile (both K-major).
+      // X^T = A_j Y^T: A_j a 128-key K/V tile, Y a 128-query Q/dO tile, both K-major.
       auto issue_t = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t ob = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_ss(tmem + d_col, sdesc_sw128(a_base + oa, 16, 1024), sdesc_sw128(b_base + ob, 16, 1024), kIdST,
+          const uint32_t off = (kk >> 2) * L::kChunk + (kk & 3) * 32;
+          mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), kIdST,
                  kk > 0);
         }
       };
-      // acc += X^T(TMEM, 64 query columns as bf16) * Y (Y a 64-row tile, MN-major)
+      // acc += X^T * Y: X^T the bf16 [128 keys][128 queries] in TMEM, written
+      // by the elementwise groups at columns a_col + 64 g + [0, 32) for query
+      // group g; Y a 128-query tile read MN-major (D contiguous).
       auto issue_acc = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + d_col, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, 8192, 1024), kIdAcc,
-                 (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + d_col, tmem + a_col + 64 * (kk >> 2) + 8 * (kk & 3),
+                 sdesc_sw128(b_base + kk * 2048, L::kChunk, 1024), kIdAcc, (acc || kk > 0) ? 1u : 0u);
       };
-      auto issue_dq = [&](int b) {
+      // dQ^T = K_j^T dS^T: K read MN-major (D contiguous), dS from the
+      // shared-memory tile, MN-major (queries contiguous).
+      auto issue_dq = [&]() {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + 128 + 64 * b, sdesc_sw128(k_addr + kk * 2048, 16384, 1024),
-                 sdesc_sw128(ds_addr + b * L::kDSTile + kk * 2048, 8192, 1024), kIdDQ, kk > 0);
+          mma_ss(tmem + t_dp, sdesc_sw128(k_addr + kk * 2048, L::kChunk, 1024),
+                 sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024), kIdDQ, kk > 0);
       };
 
-      bool ok = wait_parity(kv_full, 0, abort_flag) && (is_z || wait_parity(qd_full, 0, abort_flag));
-      if (ok && !is_z) {
-        tc_fence_after();
-        if (is_x) {
+      const int role = warp - 1;  // 0 X, 1 Y, 2 Z
+      bool ok = wait_parity(kv_full, 0, abort_flag);
+      if (role == 0) {
+        if (ok && (ok = wait_parity(q_full, 0, abort_flag))) {
+          tc_fence_after();
           issue_t(0, k_addr, q_addr);
-          mma_commit(s_full + 0);
-        } else {
-          issue_t(128, v_addr, do_addr);
-          mma_commit(dp_full + 0);
+          mma_commit(s_full);
+          mma_commit(q_empty);
+        }
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int t = it % DOS;
+          if (!(ok = wait_parity(p_full, it & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_acc(t_dv, 0, do_addr + t * L::kTile, it > 0);
+          mma_commit(do_empty + t);
+          if (it + 1 < n_it) {
+            const int ns = (it + 1) % QS;
+            if (!(ok = wait_parity(q_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_t(0, k_addr, q_addr + ns * L::kTile);  // over P^T(it): after dV(it), same thread
+            mma_commit(s_full);
+            mma_commit(q_empty + ns);
+          }
+        }
+      } else if (role == 1) {
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int s = it % QS;
+          if (!(ok = wait_parity(ds_full, it & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_acc(t_dk, t_dp, q_addr + s * L::kTile, it > 0);
+          mma_commit(q_empty + s);
+          issue_dq();  // over dS^T(it): after dK(it), same thread
+          mma_commit(dq_full);
+        }
+      } else {
+        if (ok && (ok = wait_parity(do_full, 0, abort_flag))) {
+          tc_fence_after();
+          issue_t(t_dp, v_addr, do_addr);
+          mma_commit(dp_full);
+          mma_commit(do_empty);
+        }
+        for (int it = 0; ok && it + 1 < n_it; ++it) {
+          const int nt = (it + 1) % DOS;
+          if (!(ok = wait_parity(dq_empty, it & 1, abort_flag))) break;
+          if (!(ok = wait_parity(do_full + nt, ((it + 1) / DOS) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_t(t_dp, v_addr, do_addr + nt * L::kTile);
+          mma_commit(dp_full);
+          mma_commit(do_empty + nt);
         }
       }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int b = it & 1, s = it % QS;
-        const int nb = b ^ 1, ns = (it + 1) % QS;
-        const bool has_next = it + 1 < n_it;
-        if (is_z) {
-          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_dq(b);
-          mma_commit(dq_full + b);
-        } else if (is_x) {
-          if (has_next) {
-            if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
-            if (it >= 1 && !(ok = wait_parity(y_done + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_t(64 * nb, k_addr, q_addr + ns * L::kQT);
-            mma_commit(s_full + nb);
-          }
-          if (!(ok = wait_parity(p_full + b, (it >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_acc(t_dv, 64 * b, do_addr + s * L::kQT, it > 0);
-          mma_commit(qd_empty + s);
-        } else {
-          if (has_next) {
-            if (!(ok = wait_parity(qd_full + ns, ((it + 1) / QS) & 1, abort_flag))) break;
-            if (it >= 1 && !(ok = wait_parity(dq_empty + nb, ((it - 1) >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_t(128 + 64 * nb, v_addr, do_addr + ns * L::kQT);
-            mma_commit(dp_full + nb);
-          }
-          if (!(ok = wait_parity(ds_full + b, (it >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_acc(t_dk, 64 * b + 32, q_addr + s * L::kQT, it > 0);
-          mma_commit(y_done + b);
-          mma_commit(qd_empty + s);
-        }
-      }
-      if (ok && !is_z) mma_commit(acc_full);
+      if (ok && role < 2) mma_commit(acc_full);
       // Let every MMA the issuers started finish before TMEM is freed.
       mma_commit(mma_done);
       wait_parity_drain(mma_done, 0);
     }
   } else if (wg >= 2) {
     // ---------------------------------------- elementwise (thread = key row)
-    // Group e handles iterations it = e, e+2, ... with TMEM/smem buffer b = e.
+    // Group e takes query columns [64e, 64e + 64) of every tile.
     setmaxnreg_inc<kRegElem>();
     const int e = wg - 2;
     const int quarter = warp & 3;
@@ -510,27 +558,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float lam = p.scale_log2;
     const float scale = p.scale;
-    const int b = e;
-    const uint32_t tS = tmem + lane_off + 64 * b;
-    const uint32_t tP = tmem + lane_off + 128 + 64 * b;
-    uint8_t* ds_row = smem + L::kDS + b * L::kDSTile + k * 128;
+    const uint32_t tS = tmem + lane_off + 64 * e;
+    const uint32_t tP = tmem + lane_off + t_dp + 64 * e;
+    uint8_t* ds_row = smem + L::kDS + e * (128 * 128) + k * 128;
     bool ok = true;
-    for (int it = e; it < n_it; it += 2) {
+    for (int it = 0; it < n_it; ++it) {
       const int s = it % QS;
-      const int q0 = q_start(it);
-      ok = __all_sync(0xffffffffu, wait_parity(qd_full + s, (it / QS) & 1, abort_flag) &&
-                                       wait_parity(s_full + b, (it >> 1) & 1, abort_flag));
+      const int qe = q_start(it) + 64 * e;  // first query of this group's columns
+      ok = __all_sync(0xffffffffu, wait_parity(q_full + s, (it / QS) & 1, abort_flag) &&
+                                       wait_parity(s_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const float4* lse2 = reinterpret_cast<const float4*>(smem + L::kStat + s * 512);
-      const float4* dd = lse2 + 16;
-      const bool edge = (q0 + 64 > N) || (j * 128 + 128 > N) || (MASK == kMaskCausal && j * 128 + 127 > q0) ||
-                        (MASK == kMaskBand && (j * 128 + 127 > q0 + p.wr || j * 128 < q0 + 63 - p.wl));
+      const float4* lse2 = reinterpret_cast<const float4*>(smem + L::kStat + s * 1024) + 16 * e;
+      const float4* dd = reinterpret_cast<const float4*>(smem + L::kStat + s * 1024 + 512) + 16 * e;
+      const bool edge = (qe + 64 > N) || (j * 128 + 128 > N) || (MASK == kMaskCausal && j * 128 + 127 > qe) ||
+                        (MASK == kMaskBand && (j * 128 + 127 > qe + p.wr || j * 128 < qe + 63 - p.wl));
       float pr[64];
       {
         uint32_t sv[64];
-        tmem_ld32(tS, sv);
-        tmem_ld32(tS + 32, sv + 32);
+        tmem_ld64(tS, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
@@ -544,7 +590,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (edge) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const int qi = q0 + c;
+          const int qi = qe + c;
           const bool vis = (qi < N) && (kj < N) && (MASK != kMaskCausal || kj <= qi) &&
                            (MASK != kMaskBand || (kj >= qi - p.wl && kj <= qi + p.wr));
           if (!vis) pr[c] = 0.f;
@@ -554,16 +600,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-        tmem_st32(tS, pk);
+        tmem_st32(tS, pk);  // P^T over this thread's own S^T columns
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + b);
+      if (lane == 0) mbar_arrive(p_full);
 
-      // dS tile b was last read by dQ^T(it - 2), which finished before the
-      // drain released its TMEM buffer and so before dP^T(it) was issued.
-      ok = __all_sync(0xffffffffu, wait_parity(dp_full + b, (it >> 1) & 1, abort_flag));
+      // The dS tile was last read by dQ^T(it - 1), which finished before the
+      // drain released dQ^T's TMEM and so before dP^T(it) was issued.
+      ok = __all_sync(0xffffffffu, wait_parity(dp_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -576,16 +622,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c4 = 0; c4 < 8; ++c4) {
           const float4 d4 = dd[8 * h + c4];
           const int q = 32 * h + 4 * c4;
-          const float s0 = pr[q + 0] * (__uint_as_float(dp[4 * c4 + 0]) - d4.x) * scale;
-          const float s1 = pr[q + 1] * (__uint_as_float(dp[4 * c4 + 1]) - d4.y) * scale;
-          const float s2 = pr[q + 2] * (__uint_as_float(dp[4 * c4 + 2]) - d4.z) * scale;
-          const float s3 = pr[q + 3] * (__uint_as_float(dp[4 * c4 + 3]) - d4.w) * scale;
-          pk[2 * c4] = pack_bf16(s0, s1);
-          pk[2 * c4 + 1] = pack_bf16(s2, s3);
+          const float g0 = pr[q + 0] * (__uint_as_float(dp[4 * c4 + 0]) - d4.x) * scale;
+          const float g1 = pr[q + 1] * (__uint_as_float(dp[4 * c4 + 1]) - d4.y) * scale;
+          const float g2 = pr[q + 2] * (__uint_as_float(dp[4 * c4 + 2]) - d4.z) * scale;
+          const float g3 = pr[q + 3] * (__uint_as_float(dp[4 * c4 + 3]) - d4.w) * scale;
+          pk[2 * c4] = pack_bf16(g0, g1);
+          pk[2 * c4 + 1] = pack_bf16(g2, g3);
         }
-        tmem_st16(tS + 32 + 16 * h, pk);
-        // Row k of the [128 keys][64 queries] dS tile, 128-byte swizzle:
-        // 16-byte chunk c (queries 8c..8c+7) lives at chunk c ^ (k & 7).
+        // dS^T over dP^T columns this thread has already read.
+        tmem_st16(tP + 16 * h, pk);
+        // Row k of the [128 keys][64 queries] dS group tile, 128-byte
+        // swizzle: 16-byte chunk c (queries 8c..8c+7) lives at chunk c ^ (k & 7).
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int chunk = 4 * h + c;
@@ -597,50 +644,105 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full + b);
+      if (lane == 0) mbar_arrive(ds_full);
     }
-    // -------------------------------------- epilogue: group 0 dV, group 1 dK
+    // ------------------------------ epilogue: group 0 writes dV, group 1 dK
+    // Each warp stages its 32 key rows in shared memory (128-byte swizzle)
+    // and writes them with TMA: a bf16 store, or, when CTAs share a K/V
+    // head's query heads, an fp32 reduce-add into the accumulator. Rows a
+    // TMA store cannot clip (past the end of a packed sequence) are written
+    // by the threads.
     if (ok) {
       ok = __all_sync(0xffffffffu, wait_parity(acc_full, 0, abort_flag));
       if (ok) {
         tc_fence_after();
-        const bool valid = kj < N;
-        const int kv = valid ? kj : 0;
-        // dK/dV row of key kj, in units of D elements.
-        const size_t row = packed ? static_cast<size_t>(s0 + kv) * p.Hkv + kvh : static_cast<size_t>(bkv) * N + kv;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e ? p.dk : p.dv) + row * D;
-        float* acc = (e ? p.dk_acc : p.dv_acc) + row * D;
+        const bool split = p.n_split > 1;
+        const int r0 = j * 128 + quarter * 32;  // this warp's first key
         const uint32_t col = e ? t_dk : t_dv;
+        const CUtensorMap* tm_out = e ? &tm_dk : &tm_dv;
+        if (r0 < N && (!packed || r0 + 32 <= N)) {
+          const int slot = e * 4 + quarter;
+          uint8_t* stg = smem + slot * (split ? L::kEpiF32 : L::kEpiBf16);
+          uint8_t* row = stg + lane * 128;
+          const int sw = lane & 7;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + col + c, v);
-          tmem_wait_ld();
-          if (valid && p.n_split > 1) {
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + col + 32 * c, v);
+            tmem_wait_ld();
+            if (split) {
+              // fp32 chunk c: [32 rows][32 columns = 128 B]
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              red_add_v4(acc + c + 4 * x, __uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
-                         __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
-          } else if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+              for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(row + c * 4096 + ((u ^ sw) << 4)) =
+                    make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            } else {
+              // bf16 chunk c/2: [32 rows][64 columns = 128 B], units 4(c&1)..+3
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-              dst[x] = make_uint4(pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
-                                  pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
-                                  pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
-                                  pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+              for (int x = 0; x < 4; ++x) {
+                const int u = 4 * (c & 1) + x;
+                *reinterpret_cast<uint4*>(row + (c >> 1) * 4096 + ((u ^ sw) << 4)) =
+                    make_uint4(pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                               pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                               pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                               pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (split) {
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tma_reduce_add_3d(tm_out, stg + c * 4096, 32 * c, s0 + r0, kvh);
+            } else {
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c) tma_store_3d(tm_out, stg + c * 4096, 64 * c, s0 + r0, kvh);
+            }
+            bulk_commit_group();
+            bulk_wait_group0();
+          }
+          __syncwarp();
+        } else {
+          const bool valid = kj < N;
+          const int kv = valid ? kj : 0;
+          // dK/dV row of key kj, in units of D elements.
+          const size_t orow =
+              packed ? static_cast<size_t>(s0 + kv) * p.Hkv + kvh : static_cast<size_t>(bkv) * N + kv;
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e ? p.dk : p.dv) + orow * D;
+          float* acc = (e ? p.dk_acc : p.dv_acc) + orow * D;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + col + c, v);
+            tmem_wait_ld();
+            if (valid && split) {
+#pragma unroll
+              for (int x = 0; x < 8; ++x)
+                red_add_v4(acc + c + 4 * x, __uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                           __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+            } else if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                dst[x] = make_uint4(pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                                    pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                                    pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                                    pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+            }
           }
         }
       }
     }
   } else if (wg == 1) {
     // ------------------------------------------------- dQ drain (warps 4-7)
-    // dQ_i^T sits in TMEM with the head-dim index on lanes and the 64 queries
-    // on columns. The drain copies each half (32 queries) into its own fp32
-    // [32][D] staging buffer and one TMA reduce-add per half adds it into the
-    // fp32 accumulator; the TMA engine streams the reduction to L2 while the
-    // warps stage the next half, waiting only for that buffer's previous read.
-    setmaxnreg_dec<kRegDrain>();
+    // dQ_i^T sits in TMEM with the head-dim index on lanes and the 128
+    // queries on columns. The drain copies all of it into registers and
+    // releases the TMEM at once (the next dP^T waits for that), then stages
+    // it 32 queries at a time in two fp32 [32][D] buffers; one TMA reduce-add
+    // per buffer adds it into the fp32 accumulator while the warps stage the
+    // next 32 queries.
+    setmaxnreg_inc<kRegDrain>();
     const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     // M = D = 128 uses every lane; M = 64 uses lanes 0-15 of each quarter.
@@ -648,27 +750,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool holds = (D == 128) || (lane < 16);
     const bool leader = (warp == 4 && lane == 0);
     bool ok = true;
-    // Every drain warp runs all 4*n_it named barriers, even after an abort
+    // Every drain warp runs all 8*n_it named barriers, even after an abort
     // (work is skipped instead), so no warp can be left waiting at one.
     for (int it = 0; it < n_it; ++it) {
-      const int b = it & 1;
-      if (ok) ok = __all_sync(0xffffffffu, wait_parity(dq_full + b, (it >> 1) & 1, abort_flag));
-      uint32_t v[64];
+      if (ok) ok = __all_sync(0xffffffffu, wait_parity(dq_full, it & 1, abort_flag));
+      uint32_t v[128];
       if (ok) {
         tc_fence_after();
-        tmem_ld32(tmem + lane_off + 128 + 64 * b, v);
-        tmem_ld32(tmem + lane_off + 128 + 64 * b + 32, v + 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + t_dp + 32 * c, v + 32 * c);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(dq_empty + b);
+        if (lane == 0) mbar_arrive(dq_empty);
       }
       const int q0 = q_start(it), bhq = q_head(it);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float* stg = reinterpret_cast<float*>(smem + L::kStg + h * L::kStgHalf);
-        // Groups go out in order (it-1, 0), (it-1, 1), (it, 0), ...: at most one
-        // pending means the previous read of this half's buffer is done.
+      for (int h = 0; h < 4; ++h) {
+        float* stg = reinterpret_cast<float*>(smem + L::kStg + (h & 1) * L::kStgHalf);
+        // Groups go out in order: at most one pending means the previous
+        // read of this buffer is done.
         if (leader) bulk_wait_group_read1();
         named_bar_sync(1, 128);
         if (ok && holds) {

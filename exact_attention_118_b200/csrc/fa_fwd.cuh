@@ -44,6 +44,9 @@
 // the largest e4m3 value); l sums the unrounded p.
 #pragma once
 #include <cuda.h>
+
+#include <type_traits>
+
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -82,11 +85,40 @@ struct FwdLayout {
 
 constexpr int kFwdThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Every kPolyEvery-th column pair of an unmasked tile takes its exponentials
+// on the FMA pipe (exp2_fma2) instead of the special-function unit; 0: none.
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
+
+// 2^x for a pair of fp32 values on the FMA pipe, x <= 2^22 (here x <= 8).
+// Cody and Waite's range reduction: n = round(x) by adding and subtracting
+// 1.5 * 2^23, f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) with p the degree-3
+// polynomial of least maximum relative error on [-1/2, 1/2] (Remez exchange;
+// coefficients from csrc/exp2_poly.py, relative error below 7.5e-5 in fp32),
+// and 2^n added into p's exponent field. x is clamped below at -125 so the
+// result stays a normal number (2^-125 instead of a smaller value or 0).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 t = fadd2(x, make_float2(kShift, kShift));
+  const float2 f = fsub2(x, fsub2(t, make_float2(kShift, kShift)));
+  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  // The low mantissa bits of t hold n (two's complement); shifted by 23 they
+  // land in the exponent field, and the shifter's own bits shift out.
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
 
 template <int D, int MASK, bool OF32, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams p) {
   static_assert(!FP8 || D == 128, "the FP8 forward is built for D = 128");
   constexpr int ESZ = FP8 ? 1 : 2;
   using L = FwdLayout<D, ESZ>;
@@ -104,7 +136,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* v_full = k_empty + S;
   uint64_t* v_empty = v_full + S;
   uint64_t* s_full = v_empty + S;  // [2]
-  uint64_t* p_full = s_full + 2;   // [2]
+  uint64_t* p_half = s_full + 2;   // [2] P of keys 0-63 in TMEM (and O rescaled)
+  uint64_t* p_full = p_half + 2;   // [2] P of keys 64-127 in TMEM
   uint64_t* o_full = p_full + 2;   // [2]
   uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -168,6 +201,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
+      mbar_init(p_half + t, 128);
       mbar_init(p_full + t, 128);
       mbar_init(o_full + t, 1);
     }
@@ -235,12 +269,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mma_ss(tmem + t * 128, da, db, kIdS, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int stage, bool acc) {
+      // PV over keys [64 half, 64 half + 64): the softmax hands P over in two
+      // halves, so the product over the first half overlaps the exponentials
+      // of the second.
+      auto issue_pv = [&](int t, int stage, bool acc, int half) {
         const uint32_t va = v_addr + stage * L::kTile;
         // Each MMA takes 32 bytes of P per row (8 TMEM columns: 16 bf16 or 32
         // e4m3 keys) and the matching 16 or 32 rows of V.
 #pragma unroll
-        for (int kk = 0; kk < 4 * ESZ; ++kk) {
+        for (int kk = half * 2 * ESZ; kk < (half + 1) * 2 * ESZ; ++kk) {
           const uint64_t dv = sdesc_sw128(va + kk * (32 / ESZ) * 128, 16384, 1024);
           if (FP8)
             mma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, dv, kIdO, (acc || kk > 0) ? 1u : 0u);
@@ -267,9 +304,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= a_t[t] && j < b_t[t]) {
+            if (!(ok = wait_parity(p_half + t, (j - a_t[t]) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_pv(t, s, j > a_t[t], 0);
             if (!(ok = wait_parity(p_full + t, (j - a_t[t]) & 1, abort_flag))) break;
             tc_fence_after();
-            issue_pv(t, s, j > a_t[t]);
+            issue_pv(t, s, true, 1);
             mma_commit(o_full + t);
           }
           if (t == 1) mma_commit(v_empty + s);
@@ -319,15 +359,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       }
       const int kb = (j0 + a_me + j) * 128;
+      bool masked = false;
       if (MASK == kMaskBand) {
         const int qs = q0 + 128 * t;
         if (kb + 128 > N || kb + 127 > qs + p.wr || kb < qs + 127 - p.wl) {
+          masked = true;
           const int hi = min(N - kb, qi + p.wr - kb + 1), lo = qi - p.wl - kb;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= hi || c < lo) s[c] = -INFINITY;
         }
       } else if (kb + 128 > N || (MASK == kMaskCausal && kb + 127 > q0 + 128 * t)) {
+        masked = true;
         int lim = N - kb;
         if (MASK == kMaskCausal) lim = min(lim, qi - kb + 1);
 #pragma unroll
@@ -350,47 +393,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_blk;
         rescale = true;
       }
-      // A band can hide a whole tile from some rows: while a row has seen no
-      // visible key its m is -inf and its p must come out 0, not NaN.
-      const float neg_m = (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m;
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pk[64];
-      if (FP8) {
-        // Four e4m3 probabilities per TMEM column: P fills 32 columns.
-        const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
-        float2 rs = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float2 x0 = ffma2(make_float2(s[4 * c], s[4 * c + 1]), lam2, negm2);
-          const float2 x1 = ffma2(make_float2(s[4 * c + 2], s[4 * c + 3]), lam2, negm2);
-          const float2 p01 = make_float2(ex2(x0.x), ex2(x0.y)), p23 = make_float2(ex2(x1.x), ex2(x1.y));
-          rs = fadd2(rs, p01);
-          rs = fadd2(rs, p23);
-          pk[c] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
-        }
-        rs0 = rs.x;
-        rs1 = rs.y;
-      } else {
-        const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
-        float2 rs = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), lam2, negm2);
-          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          rs = fadd2(rs, pp);
-          pk[c] = pack_bf16(pp.x, pp.y);
-        }
-        rs0 = rs.x;
-        rs1 = rs.y;
-      }
-      l = l * alpha + (rs0 + rs1);
-      tmem_st32(tS + 0, pk + 0);
-      if (!FP8) tmem_st32(tS + 32, pk + 32);
       if (j > 0) {
         // PV_{j-1} finished before S_j (same issuing thread, committed
         // earlier), so this wait is immediate; it keeps the phase count exact.
         ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (j - 1) & 1, abort_flag));
         if (!ok) break;
+        // O is rescaled before the first half of P is handed over: PV_j
+        // accumulates into it from then on.
         if (__any_sync(0xffffffffu, rescale)) {
           tc_fence_after();
 #pragma unroll
@@ -404,9 +413,61 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full + t);
+      // A band can hide a whole tile from some rows: while a row has seen no
+      // visible key its m is -inf and its p must come out 0, not NaN.
+      const float neg_m = (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m;
+      const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
+      float2 rs = make_float2(0.f, 0.f);
+      if (FP8) {
+        // Four e4m3 probabilities per TMEM column: P fills 32 columns.
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float2 x0 = ffma2(make_float2(s[4 * c], s[4 * c + 1]), lam2, negm2);
+          const float2 x1 = ffma2(make_float2(s[4 * c + 2], s[4 * c + 3]), lam2, negm2);
+          const float2 p01 = make_float2(ex2(x0.x), ex2(x0.y)), p23 = make_float2(ex2(x1.x), ex2(x1.y));
+          rs = fadd2(rs, p01);
+          rs = fadd2(rs, p23);
+          pk[c] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
+        }
+        tmem_st32(tS + 0, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_half + t);
+        mbar_arrive(p_full + t);
+      } else {
+        // Tiles without masking send some column pairs through the FMA-pipe
+        // exp2 (exp2_fma2), which takes load off the special-function unit;
+        // masked tiles keep every exponential on ex2, which gives exactly 0
+        // for -inf.
+        auto half = [&](auto use_poly, int hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            const int c = 32 * hh + cc;
+            const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), lam2, negm2);
+            float2 pp;
+            if (decltype(use_poly)::value && c % kPolyEvery == kPolyEvery - 1)
+              pp = exp2_fma2(x);
+            else
+              pp = make_float2(ex2(x.x), ex2(x.y));
+            rs = fadd2(rs, pp);
+            pk[cc] = pack_bf16(pp.x, pp.y);
+          }
+          tmem_st32(tS + 32 * hh, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(hh ? p_full + t : p_half + t);
+        };
+        if (kPolyEvery > 0 && !masked) {
+          half(std::true_type{}, 0);
+          half(std::true_type{}, 1);
+        } else {
+          half(std::false_type{}, 0);
+          half(std::false_type{}, 1);
+        }
+      }
+      l = l * alpha + (rs.x + rs.y);
     }
 
     // ------------------------------------------------------------ epilogue
@@ -421,28 +482,63 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const size_t row = packed ? static_cast<size_t>(s0 + qv) * p.H + hq : static_cast<size_t>(bh) * N + qv;
         const size_t li = packed ? static_cast<size_t>(hq) * p.T + s0 + qv : row;
         if (valid) p.lse[li] = (m + log2f(l)) * 0.69314718055994531f;
+        const int r0 = q0 + 128 * t + 32 * quarter;  // this warp's first query
+        if (!OF32 && !FP8 && r0 < N && (!packed || r0 + 32 <= N)) {
+          // bf16 O: each warp stages its 32 rows in its part of the tile's Q
+          // buffer (free: the tile's last S MMA has read it) with the 128-byte
+          // swizzle and writes them with TMA stores, which clip rows past N.
+          uint8_t* stg = smem + (t ? L::kQ1 : L::kQ0) + quarter * (32 * D * 2);
+          uint8_t* orow = stg + lane * 128;
+          const int sw = lane & 7;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + c, ov);
-          tmem_wait_ld();
-          if (valid) {
-            if (OF32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row * D + c);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l, __uint_as_float(ov[4 * e + 1]) * inv_l,
-                                     __uint_as_float(ov[4 * e + 2]) * inv_l, __uint_as_float(ov[4 * e + 3]) * inv_l);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D + c);
+            for (int x = 0; x < 4; ++x) {
+              const int u = 4 * (c & 1) + x;
+              *reinterpret_cast<uint4*>(orow + (c >> 1) * 4096 + ((u ^ sw) << 4)) = make_uint4(
+                  pack_bf16(__uint_as_float(ov[8 * x + 0]) * inv_l, __uint_as_float(ov[8 * x + 1]) * inv_l),
+                  pack_bf16(__uint_as_float(ov[8 * x + 2]) * inv_l, __uint_as_float(ov[8 * x + 3]) * inv_l),
+                  pack_bf16(__uint_as_float(ov[8 * x + 4]) * inv_l, __uint_as_float(ov[8 * x + 5]) * inv_l),
+                  pack_bf16(__uint_as_float(ov[8 * x + 6]) * inv_l, __uint_as_float(ov[8 * x + 7]) * inv_l));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint4 w;
-                w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
-                w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
-                w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
-                w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
-                dst[e] = w;
+            for (int c = 0; c < D / 64; ++c) tma_store_3d(&tm_o, stg + c * 4096, 64 * c, s0 + r0, hq);
+            bulk_commit_group();
+            bulk_wait_group0();
+          }
+          __syncwarp();
+        } else {
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c, ov);
+            tmem_wait_ld();
+            if (valid) {
+              if (OF32) {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row * D + c);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l, __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                       __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                       __uint_as_float(ov[4 * e + 3]) * inv_l);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D + c);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  uint4 w;
+                  w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                  w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                  w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                  w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                  dst[e] = w;
+                }
               }
             }
           }

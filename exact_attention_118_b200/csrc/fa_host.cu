@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -12,6 +13,10 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+
+static_assert(fa::kDevErrTimeout == FA_DEVERR_TIMEOUT && fa::kDevErrSmemAlign == FA_DEVERR_SMEM_ALIGN &&
+                  fa::kDevErrSeqlens == FA_DEVERR_SEQLENS,
+              "device error bits must match the header");
 
 namespace {
 
@@ -34,6 +39,103 @@ EncodeTiledFn encode_fn() {
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   });
   return g_encode;
+}
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+// The unique ID of the CUDA context current on this thread, 0 if there is
+// none. The driver never reuses a context ID within a process, so state kept
+// under one ID is never taken for state of a later context (one created after
+// cudaDeviceReset, or one the caller made current through the driver API).
+unsigned long long current_ctx_id() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  if (!g_ctx_current || !g_ctx_id) return 0;
+  CUcontext c = nullptr;
+  if (g_ctx_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  return g_ctx_id(c, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// A small table of values kept per CUDA context: the results of one-time
+// set-up steps. Up to kSlots contexts; past that the oldest entry is reused.
+template <typename T>
+class PerContext {
+ public:
+  bool get(unsigned long long id, T* out) {
+    if (id == 0) return false;
+    std::lock_guard<std::mutex> lock(mu_);
+    for (int i = 0; i < n_; ++i)
+      if (ids_[i] == id) {
+        *out = vals_[i];
+        return true;
+      }
+    return false;
+  }
+  void put(unsigned long long id, T v) {
+    if (id == 0) return;
+    std::lock_guard<std::mutex> lock(mu_);
+    for (int i = 0; i < n_; ++i)
+      if (ids_[i] == id) {
+        vals_[i] = v;
+        return;
+      }
+    const int slot = n_ < kSlots ? n_++ : (next_++ % kSlots);
+    ids_[slot] = id;
+    vals_[slot] = v;
+  }
+
+ private:
+  static constexpr int kSlots = 16;
+  std::mutex mu_;
+  unsigned long long ids_[kSlots] = {};
+  T vals_[kSlots] = {};
+  int n_ = 0, next_ = 0;
+};
+
+// A kernel's dynamic shared memory limit is raised once per context, not on
+// every launch. The caller keeps one table per kernel instantiation.
+template <typename Kern>
+fa_status set_smem_once(PerContext<int>& done, Kern kern, int smem) {
+  int have = 0;
+  if (done.get(current_ctx_id(), &have) && have == smem) return FA_OK;
+  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) {
+    t_last_cuda_error = static_cast<int>(e);
+    return FA_ERR_CUDA;
+  }
+  done.put(current_ctx_id(), smem);  // the call above makes a context current if none was
+  return FA_OK;
+}
+
+constexpr int kMaxDevices = 64;
+
+// Streaming multiprocessors of the current device, cached per device.
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  if (slot) cache[dev].store(sms, std::memory_order_relaxed);
+  return sms;
 }
 
 // The kernels use tcgen05 and TMA: compute capability 10.0 (sm_100a) only.
@@ -100,6 +202,13 @@ fa_status make_bf16_tile_map(CUtensorMap* m, const void* base, const Geom& g, in
                        CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// bf16 output rows in 32-row boxes of 64 columns (128-byte swizzle): the
+// per-warp TMA stores of O, dK and dV.
+fa_status make_out_map(CUtensorMap* m, const void* base, const Geom& g, int heads, int d) {
+  return make_head_map(m, base, g, heads, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, 64, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Caller-provided events recorded around the main backward kernel
 // (fa_set_bwd_main_events); per host thread.
 thread_local cudaEvent_t t_bwd_ev_before = nullptr;
@@ -120,13 +229,7 @@ fa_status cuda_fail(cudaError_t e) {
 // Grid for the memory-bound helper kernels: enough CTAs to fill every SM a
 // few times over, grid-striding beyond that.
 unsigned helper_grid(long long threads_needed) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  const int sms = sm_count();
   const long long blocks = (threads_needed + 255) / 256;
   const long long cap = static_cast<long long>(sms) * 8;
   return static_cast<unsigned>(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
@@ -144,10 +247,7 @@ unsigned helper_grid(long long threads_needed) {
 // heaviest-first order. Returns the number of groups.
 int sched_groups(long long bytes_per_unit, int units, int tiles) {
   if (bytes_per_unit * units <= (256ll << 20)) return 1;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                 cudaSuccess)
-    sms = 148;
+  const int sms = sm_count();
   const long long budget = 64ll << 20;
   long long g_max = bytes_per_unit > 0 ? budget / bytes_per_unit : units;
   if (g_max < 1) g_max = 1;
@@ -177,33 +277,33 @@ Mask resolve_mask(int wl, int wr, int N) {
 }
 
 template <int D, int MASK, bool OF32, bool FP8 = false>
-fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
-                     cudaStream_t st) {
+fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                     const fa::FwdParams& p, cudaStream_t st) {
   auto kern = fa::fa_fwd_kernel<D, MASK, OF32, FP8>;
   const int smem = fa::FwdLayout<D, FP8 ? 1 : 2>::kAlloc;
-  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
-    return cuda_fail(e);
+  static PerContext<int> attr_set;
+  if (fa_status s = set_smem_once(attr_set, kern, smem)) return s;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
-  kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, p);
+  kern<<<grid, fa::kFwdThreads, smem, st>>>(tq, tk, tv, to, p);
   return launch_status();
 }
 
 template <int D, bool OF32, bool FP8 = false>
-fa_status launch_fwd_mask(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+fa_status launch_fwd_mask(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                           const fa::FwdParams& p, int mode, cudaStream_t st) {
-  if (mode == fa::kMaskCausal) return launch_fwd<D, fa::kMaskCausal, OF32, FP8>(tq, tk, tv, p, st);
-  if (mode == fa::kMaskBand) return launch_fwd<D, fa::kMaskBand, OF32, FP8>(tq, tk, tv, p, st);
-  return launch_fwd<D, fa::kMaskNone, OF32, FP8>(tq, tk, tv, p, st);
+  if (mode == fa::kMaskCausal) return launch_fwd<D, fa::kMaskCausal, OF32, FP8>(tq, tk, tv, to, p, st);
+  if (mode == fa::kMaskBand) return launch_fwd<D, fa::kMaskBand, OF32, FP8>(tq, tk, tv, to, p, st);
+  return launch_fwd<D, fa::kMaskNone, OF32, FP8>(tq, tk, tv, to, p, st);
 }
 
 // 2-D fp32 map of a [BH][Np] statistics array (Np >= N, a multiple of 4),
-// dims {N, BH}: a 64-wide row box, zero-filled past N.
+// dims {N, BH}: a 128-wide row box (one query tile), zero-filled past N.
 fa_status make_stat_map(CUtensorMap* m, const float* base, int N, int Np, int BH) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FA_ERR_CUDA;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Np) * 4};
-  const cuuint32_t box[2] = {64u, 1u};
+  const cuuint32_t box[2] = {128u, 1u};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -216,11 +316,12 @@ template <int D, int MASK>
 fa_status launch_bwd_main(const CUtensorMap* maps, const fa::BwdParams& p, cudaStream_t st) {
   auto kern = fa::fa_bwd_kernel<D, MASK>;
   const int smem = fa::BwdLayout<D>::kAlloc;
-  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
-    return cuda_fail(e);
+  static PerContext<int> attr_set;
+  if (fa_status s = set_smem_once(attr_set, kern, smem)) return s;
   const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
   if (t_bwd_ev_before && cudaEventRecord(t_bwd_ev_before, st) != cudaSuccess) return FA_ERR_CUDA;
-  kern<<<grid, fa::kBwdThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p);
+  kern<<<grid, fa::kBwdThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7],
+                                            maps[8], p);
   const fa_status s = launch_status();
   if (s == FA_OK && t_bwd_ev_after && cudaEventRecord(t_bwd_ev_after, st) != cudaSuccess) return FA_ERR_CUDA;
   return s;
@@ -236,10 +337,7 @@ fa_status launch_bwd_main(const CUtensorMap* maps, const fa::BwdParams& p, cudaS
 int bwd_split(int B, int H, int Hkv, int N) {
   const int group = H / Hkv;
   if (group == 1) return 1;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                 cudaSuccess)
-    sms = 148;
+  const int sms = sm_count();
   const long long base = static_cast<long long>((N + 127) / 128) * B * Hkv;
   for (int s = 1; s < group; ++s)
     if (group % s == 0 && base * s >= 8LL * sms) return s;
@@ -291,22 +389,27 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   fa_status s = launch_status();
   if (s != FA_OK) return s;
 
-  // 2. Main kernel. Maps: q, k, v, dO, dQ accumulator (fp32, 32-row box), lse2, D.
-  alignas(64) CUtensorMap maps[7];
-  if ((s = make_head_map(&maps[0], q, g, g.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, 64, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
-    return s;
+  // 2. Main kernel. Maps: q, k, v, dO (128-row tiles), dQ accumulator (fp32,
+  // 32-row box), lse2, D, and the dK, dV outputs (32-row boxes; bf16, or the
+  // fp32 accumulators when query heads are split across CTAs).
+  alignas(64) CUtensorMap maps[9];
+  if ((s = make_bf16_tile_map(&maps[0], q, g, g.H, D)) != FA_OK) return s;
   if ((s = make_bf16_tile_map(&maps[1], k, g, g.Hkv, D)) != FA_OK) return s;
   if ((s = make_bf16_tile_map(&maps[2], v, g, g.Hkv, D)) != FA_OK) return s;
-  if ((s = make_head_map(&maps[3], dO, g, g.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, 64, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
-    return s;
+  if ((s = make_bf16_tile_map(&maps[3], dO, g, g.H, D)) != FA_OK) return s;
   if ((s = make_head_map(&maps[4], dq_acc, g, g.H, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, D, 32,
                          CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return s;
   const int stat_dim = g.packed() ? Np : Nr;
   if ((s = make_stat_map(&maps[5], lse2, stat_dim, Np, BHr)) != FA_OK) return s;
   if ((s = make_stat_map(&maps[6], dsum, stat_dim, Np, BHr)) != FA_OK) return s;
+  for (int t = 0; t < 2; ++t) {
+    const void* out = n_split > 1 ? static_cast<const void*>(t ? dv_acc : dk_acc) : (t ? dv : dk);
+    s = n_split > 1 ? make_head_map(&maps[7 + t], out, g, g.Hkv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, 32, 32,
+                                    CU_TENSOR_MAP_SWIZZLE_128B)
+                    : make_out_map(&maps[7 + t], out, g, g.Hkv, D);
+    if (s != FA_OK) return s;
+  }
   fa::BwdParams p;
   p.dk = dk;
   p.dv = dv;
@@ -347,7 +450,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
 
 // Failure-detection self-test: one thread waits, through the same bounded
 // wait the kernels use, on an mbarrier that nothing ever completes. The wait
-// gives up after its time limit, records FA_DEVERR_TIMEOUT in the device error
+// gives up after its time limit, records a timeout in the device error
 // word and the kernel returns normally.
 __global__ void fa_selftest_wait_kernel() {
   __shared__ uint64_t bar;
@@ -368,25 +471,23 @@ __global__ void fa_selftest_wait_kernel() {
 // backward's workspace lives in this file-scope device array instead. Every
 // GPU that loads the library holds it (FA_NOALLOC_SCRATCH_BYTES) until exit.
 // In host code the array's name is only a stand-in, not a device address:
-// its address on each device comes from cudaGetSymbolAddress, taken once per
-// device with that device current and cached here.
+// its address comes from cudaGetSymbolAddress, taken with the device current
+// and cached per CUDA context. The address belongs to the context, so a new
+// context on the same device (after cudaDeviceReset, or a driver-API context
+// the caller made current) takes its own.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+PerContext<void*> g_noalloc_addr;
 
 fa_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
-  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* addr = nullptr;
-    if (cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch)) return cuda_fail(e);
-    g_noalloc_addr[dev] = addr;
+  void* addr = nullptr;
+  if (g_noalloc_addr.get(current_ctx_id(), &addr) && addr != nullptr) {
+    *out = addr;
+    return FA_OK;
   }
-  *out = g_noalloc_addr[dev];
+  if (cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch)) return cuda_fail(e);
+  g_noalloc_addr.put(current_ctx_id(), addr);  // the lookup makes a context current if none was
+  *out = addr;
   return FA_OK;
 }
 
@@ -394,10 +495,13 @@ fa_status noalloc_scratch(void** out) {
 fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, void* o, float* lse, int d,
                    float scale, int window_left, int window_right, fa_dtype o_dtype, void* stream) {
   fa_status s;
-  alignas(64) CUtensorMap tq, tk, tv;
+  alignas(64) CUtensorMap tq, tk, tv, to;
   if ((s = make_bf16_tile_map(&tq, q, g, g.H, d)) != FA_OK) return s;
   if ((s = make_bf16_tile_map(&tk, k, g, g.Hkv, d)) != FA_OK) return s;
   if ((s = make_bf16_tile_map(&tv, v, g, g.Hkv, d)) != FA_OK) return s;
+  // bf16 O, stored by TMA in 32-row boxes (an fp32 O is written by the
+  // threads; the map is then unused).
+  if ((s = make_out_map(&to, o, g, g.H, d)) != FA_OK) return s;
 
   fa::FwdParams p;
   p.o = o;
@@ -418,10 +522,10 @@ fa_status fwd_impl(const Geom& g, const void* q, const void* k, const void* v, v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool f32 = (o_dtype == FA_F32);
   if (d == 64)
-    return f32 ? launch_fwd_mask<64, true>(tq, tk, tv, p, m.mode, st)
-               : launch_fwd_mask<64, false>(tq, tk, tv, p, m.mode, st);
-  return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, p, m.mode, st)
-             : launch_fwd_mask<128, false>(tq, tk, tv, p, m.mode, st);
+    return f32 ? launch_fwd_mask<64, true>(tq, tk, tv, to, p, m.mode, st)
+               : launch_fwd_mask<64, false>(tq, tk, tv, to, p, m.mode, st);
+  return f32 ? launch_fwd_mask<128, true>(tq, tk, tv, to, p, m.mode, st)
+             : launch_fwd_mask<128, false>(tq, tk, tv, to, p, m.mode, st);
 }
 
 // The FP8 forward (fixed-length layout, D = 128); arguments already checked.
@@ -429,8 +533,9 @@ fa_status fwd_fp8_impl(const Geom& g, const void* q8, const void* k8, const void
                        float scale, float q_scale, float k_scale, float v_scale, int window_left, int window_right,
                        fa_dtype o_dtype, void* stream) {
   fa_status s;
-  alignas(64) CUtensorMap tq, tk, tv;
+  alignas(64) CUtensorMap tq, tk, tv, to;
   const auto u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if ((s = make_out_map(&to, o, g, g.H, 128)) != FA_OK) return s;  // unused: the FP8 kernel's threads write O
   if ((s = make_head_map(&tq, q8, g, g.H, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
   if ((s = make_head_map(&tk, k8, g, g.Hkv, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
   if ((s = make_head_map(&tv, v8, g, g.Hkv, u8, 1, 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK) return s;
@@ -451,8 +556,8 @@ fa_status fwd_fp8_impl(const Geom& g, const void* q8, const void* k8, const void
   p.cu_seqlens = g.cu;
   p.T = g.T;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return o_dtype == FA_F32 ? launch_fwd_mask<128, true, true>(tq, tk, tv, p, m.mode, st)
-                           : launch_fwd_mask<128, false, true>(tq, tk, tv, p, m.mode, st);
+  return o_dtype == FA_F32 ? launch_fwd_mask<128, true, true>(tq, tk, tv, to, p, m.mode, st)
+                           : launch_fwd_mask<128, false, true>(tq, tk, tv, to, p, m.mode, st);
 }
 
 // The backward for either layout; arguments already checked.
@@ -476,6 +581,18 @@ fa_status check_varlen(const int* cu_seqlens, int B, int max_seqlen, int T, int 
   if (static_cast<long long>(B) * H >= (1ll << 31)) return FA_ERR_INVALID_ARG;
   if ((static_cast<long long>(T) + 4LL * B + 8) * H >= (1ll << 31)) return FA_ERR_INVALID_ARG;
   return FA_OK;
+}
+
+// Test hook: y = exp2_fma2(x), the forward's FMA-pipe exp2, element by
+// element (pairs; an odd last element is paired with itself).
+__global__ void fa_selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = 2 * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x); i < n; i += 2 * stride) {
+    const bool pair = i + 1 < n;
+    const float2 r = fa::exp2_fma2(make_float2(x[i], pair ? x[i + 1] : x[i]));
+    y[i] = r.x;
+    if (pair) y[i + 1] = r.y;
+  }
 }
 
 }  // namespace
@@ -624,25 +741,38 @@ fa_status fa_selftest_wait_timeout(void* stream) {
   return launch_status();
 }
 
+fa_status fa_selftest_exp2_fma(const float* x, float* y, long long n, void* stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  fa_status s = check_device();
+  if (s != FA_OK) return s;
+  fa_selftest_exp2_kernel<<<helper_grid((n + 1) / 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
+}
+
 fa_status fa_set_bwd_main_events(void* before, void* after) {
   t_bwd_ev_before = static_cast<cudaEvent_t>(before);
   t_bwd_ev_after = static_cast<cudaEvent_t>(after);
   return FA_OK;
 }
 
+fa_status fa_decode_device_error(unsigned int word) {
+  if (word == 0u) return FA_OK;
+  if (word & FA_DEVERR_TIMEOUT) return FA_ERR_TIMEOUT;
+  if (word & ~FA_DEVERR_SEQLENS) return FA_ERR_CUDA;  // FA_DEVERR_SMEM_ALIGN or an unknown bit
+  return FA_ERR_INVALID_ARG;                               // malformed cu_seqlens, clamped by the kernels
+}
+
 fa_status fa_get_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaError_t e = cudaStreamSynchronize(st)) return cuda_fail(e);
   unsigned int word = 0u;
-  if (cudaMemcpyFromSymbol(&word, fa::g_device_error, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaError_t e = cudaMemcpyFromSymbol(&word, fa::g_device_error, sizeof(word))) return cuda_fail(e);
   if (word != 0u) {
     const unsigned int zero = 0u;
-    if (cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-    // Only malformed cu_seqlens: a caller error that the kernels clamped.
-    if (word == fa::FA_DEVERR_SEQLENS) return FA_ERR_INVALID_ARG;
-    return FA_ERR_TIMEOUT;
+    if (cudaError_t e = cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(zero))) return cuda_fail(e);
   }
-  return FA_OK;
+  return fa_decode_device_error(word);
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,

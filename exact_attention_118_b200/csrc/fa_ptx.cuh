@@ -2,7 +2,7 @@
 // waits, TMA tensor copies, tcgen05 MMA/TMEM, and shared-memory descriptors.
 //
 // Every wait in this library goes through wait_parity(), which gives up after
-// kWaitLimitNs of wall time (read from %globaltimer), records FA_DEVERR_TIMEOUT
+// kWaitLimitNs of wall time (read from %globaltimer), records kDevErrTimeout
 // in the device error word and raises a CTA-wide abort flag in shared memory,
 // so that every role leaves its loop and the CTA can free its TMEM and exit.
 #pragma once
@@ -14,10 +14,12 @@ namespace fa {
 
 // ---------------------------------------------------------------- error word
 // The library is a single translation unit, so the word is defined here.
+// Its bits are the FA_DEVERR_* values of the C header (fa_host.cu checks that
+// the two agree).
 __device__ unsigned int g_device_error = 0u;
-constexpr unsigned int FA_DEVERR_TIMEOUT = 1u;
-constexpr unsigned int FA_DEVERR_SMEM_ALIGN = 2u;  // dynamic shared memory not 1 KB aligned
-constexpr unsigned int FA_DEVERR_SEQLENS = 4u;     // cu_seqlens entries outside [0, T] or not increasing
+constexpr unsigned int kDevErrTimeout = 1u;
+constexpr unsigned int kDevErrSmemAlign = 2u;  // dynamic shared memory not 1 KB aligned
+constexpr unsigned int kDevErrSeqlens = 4u;    // cu_seqlens entries outside [0, T] or not increasing
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -74,7 +76,7 @@ __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, vola
     if ((++polls & 255u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
-        atomicOr(&g_device_error, FA_DEVERR_TIMEOUT);
+        atomicOr(&g_device_error, kDevErrTimeout);
         *abort_flag = 1;
         return false;
       }
@@ -91,7 +93,7 @@ __device__ __forceinline__ void wait_parity_drain(uint64_t* bar, uint32_t parity
   uint32_t polls = 0;
   while (!mbar_try_wait(a, parity)) {
     if ((++polls & 255u) == 0u && globaltimer() - t0 > kWaitLimitNs / 4) {
-      atomicOr(&g_device_error, FA_DEVERR_TIMEOUT);
+      atomicOr(&g_device_error, kDevErrTimeout);
       return;
     }
   }
@@ -388,11 +390,11 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // its length L, from the prefix sums cu[b] and cu[b + 1]. Entries that would
 // reach outside the T packed rows, run backwards or exceed max_len are
 // clamped, so no access leaves the caller's buffers, and recorded as
-// FA_DEVERR_SEQLENS.
+// kDevErrSeqlens.
 __device__ __forceinline__ void seq_range(const int* cu, int b, int T, int max_len, int& s0, int& L) {
   const int a = __ldg(cu + b), e = __ldg(cu + b + 1);
   if ((a < 0 || e < a || e > T || e - a > max_len) && threadIdx.x == 0)
-    atomicOr(&g_device_error, FA_DEVERR_SEQLENS);
+    atomicOr(&g_device_error, kDevErrSeqlens);
   s0 = min(max(a, 0), T);
   L = min(min(max(e, s0), T) - s0, max_len);
 }

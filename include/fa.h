@@ -25,9 +25,11 @@
  *   Pointers   device pointers (CUDA global memory of the current device),
  *              each 16-byte aligned. The caller owns every buffer, including
  *              the backward workspace. The library allocates no device memory
- *              at run time. Across calls it keeps only the per-device address
- *              of fa_bwd_noalloc's fixed scratch array (part of the loaded
- *              module) and, per host thread, the last CUDA error code.
+ *              at run time. Across calls it keeps, per CUDA context, the
+ *              address of fa_bwd_noalloc's fixed scratch array (part of the
+ *              loaded module) and which kernels have had their shared-memory
+ *              limit raised; per device, the SM count; and, per host thread,
+ *              the last CUDA error code.
  *   Sizes      B >= 1, H >= 1, N >= 1 (any value, ragged tails are handled),
  *              d in {64, 128}, B*H*N < 2^31, N <= 2^29 (T <= 2^29 packed).
  *   scale      the factor applied to Q K^T (1/sqrt(d) in the pages' pseudocode,
@@ -43,7 +45,8 @@
  *              returns FA_ERR_CUDA. Every device-side wait in the kernels has
  *              a time limit; if one gives up, the kernel records it in a
  *              device error word and returns early, and fa_get_device_error
- *              reports FA_ERR_TIMEOUT.
+ *              reports FA_ERR_TIMEOUT (fa_decode_device_error lists every
+ *              bit of that word and its status).
  */
 #ifndef FA_B200_H
 #define FA_B200_H
@@ -119,9 +122,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * launch. No call allocates: no cudaMalloc, cudaFree or allocating library
  * routine.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture. Every call shares the one array and
+ * The first call in each CUDA context (normally one per device: the
+ * device's primary context) looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it under the
+ * context's unique ID, so a context created later - after cudaDeviceReset,
+ * or one the caller makes current through the driver API - looks it up
+ * afresh instead of reusing a stale address. Make that first call before any
+ * stream capture. Every call shares the one array and
  * the array keeps the last call's contents (the call itself clears what must
  * start at zero), so calls whose work overlaps on the GPU - on different
  * streams, or from different threads - race on it: order them on one stream
@@ -242,13 +249,30 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, fl
                      int window_left, int window_right, fa_dtype o_dtype, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device error word.
- * Returns FA_ERR_TIMEOUT if any kernel of this library gave up a bounded wait
- * since the last call, FA_ERR_INVALID_ARG if the only thing recorded is a
- * malformed cu_seqlens array (variable-length calls), FA_ERR_CUDA if the
- * synchronisation failed, else FA_OK.
+ * Synchronises `stream`, then reads and clears the device error word and
+ * returns fa_decode_device_error of it: FA_OK if nothing was recorded since
+ * the last call. FA_ERR_CUDA also if the synchronisation or the read failed.
  */
 fa_status fa_get_device_error(void* stream);
+
+/*
+ * Bits of the device error word that the kernels set (the word is the OR of
+ * everything recorded since it was last cleared).
+ */
+#define FA_DEVERR_TIMEOUT 1u    /* a bounded wait gave up; the kernel returned early */
+#define FA_DEVERR_SMEM_ALIGN 2u /* dynamic shared memory was not 1 KB aligned; the kernel did nothing */
+#define FA_DEVERR_SEQLENS 4u    /* cu_seqlens entries outside [0, T], decreasing, or longer than max_seqlen */
+
+/*
+ * The status a device error word stands for (host only, no CUDA call), in
+ * this order of precedence: 0 -> FA_OK; any FA_DEVERR_TIMEOUT ->
+ * FA_ERR_TIMEOUT; else FA_DEVERR_SMEM_ALIGN or any bit not listed above ->
+ * FA_ERR_CUDA (the launch environment broke a kernel's assumption, no result
+ * was computed); else (FA_DEVERR_SEQLENS alone) -> FA_ERR_INVALID_ARG (the
+ * kernels clamped the malformed prefix sums; results for those sequences are
+ * unspecified).
+ */
+fa_status fa_decode_device_error(unsigned int word);
 
 /*
  * Measurement hook. After this call, every fa_bwd made by the calling host
@@ -277,6 +301,15 @@ int fa_last_cuda_error(void);
  * Returns FA_OK once launched.
  */
 fa_status fa_selftest_wait_timeout(void* stream);
+
+/*
+ * Test hook for the forward kernel's exp2 on the FMA pipe (Cody-Waite range
+ * reduction and a fitted cubic; see fa_fwd.cuh): y[i] = 2^x[i] for n fp32
+ * device values, as the softmax computes it for part of its exponentials.
+ * Asynchronous on `stream`. FA_ERR_INVALID_ARG for n < 0 or null pointers
+ * with n > 0.
+ */
+fa_status fa_selftest_exp2_fma(const float* x, float* y, long long n, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* fa_strerror(fa_status status);

@@ -14,10 +14,12 @@ FAKE = 1 << 20  # an aligned, non-null address that is never dereferenced
 def test_library_loads_and_exports_every_header_symbol():
     names = fa.header_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_noalloc", "fa_get_device_error",
+                          "fa_decode_device_error",
                           "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_gqa_workspace_size",
                           "fa_fwd_window", "fa_bwd_window", "fa_fwd_varlen", "fa_bwd_varlen",
                           "fa_bwd_varlen_workspace_size", "fa_fwd_fp8",
                           "fa_set_bwd_main_events", "fa_last_cuda_error", "fa_selftest_wait_timeout",
+                          "fa_selftest_exp2_fma",
                           "fa_strerror", "fa_version"}
     lib = ctypes.CDLL(fa.LIB_PATH)
     for n in names:
@@ -30,6 +32,36 @@ def test_strerror_and_version():
         assert fa.fa_strerror(s) and fa.fa_strerror(s) != "success"
     assert fa.fa_strerror(99) == "unknown status"
     assert fa.fa_version() >= 100
+
+
+@pytest.mark.parametrize("word", range(16))
+def test_device_error_word_decoding(word):
+    # Every combination of the three defined bits and one undefined bit (8):
+    # a timeout wins; then a misaligned shared-memory window or an unknown
+    # bit (a broken launch environment, nothing computed) is a CUDA error;
+    # malformed cu_seqlens alone is the caller's argument error.
+    got = fa.fa_decode_device_error(word)
+    if word == 0:
+        want = fa.FA_OK
+    elif word & fa.FA_DEVERR_TIMEOUT:
+        want = fa.FA_ERR_TIMEOUT
+    elif word & (fa.FA_DEVERR_SMEM_ALIGN | 8):
+        want = fa.FA_ERR_CUDA
+    else:
+        assert word == fa.FA_DEVERR_SEQLENS
+        want = fa.FA_ERR_INVALID_ARG
+    assert got == want, (word, got, want)
+    assert fa.fa_decode_device_error(0x80000000 | fa.FA_DEVERR_SEQLENS) == fa.FA_ERR_CUDA
+
+
+def test_device_error_bits_match_header():
+    import re
+
+    with open(fa.HEADER_PATH) as f:
+        text = f.read()
+    bits = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (FA_DEVERR_\w+) (\d+)u", text)}
+    assert bits == {"FA_DEVERR_TIMEOUT": fa.FA_DEVERR_TIMEOUT, "FA_DEVERR_SMEM_ALIGN": fa.FA_DEVERR_SMEM_ALIGN,
+                    "FA_DEVERR_SEQLENS": fa.FA_DEVERR_SEQLENS}
 
 
 def test_workspace_size():

@@ -6,9 +6,11 @@ a latency-critical path where an allocation's unpredictable cost is not
 allowed. fa_bwd_noalloc serves them by keeping the backward's scratch in one
 fixed device array inside the library instead of a caller-owned workspace.
 
-This test calls it through the C ABI twice in a row, on different problems,
-and checks each result against fa_bwd (the entry point with a caller-owned
-workspace) within the gradient tolerance the parity tests use. The second
+This test calls it through the C ABI twice in a row, on different problems.
+It runs the same kernels as fa_bwd (the entry point with a caller-owned
+workspace), so dK and dV must equal fa_bwd's bit for bit; dQ is summed with
+fp32 adds whose order may differ between runs, so it is checked against the
+fp64 oracle within the gradient tolerance the parity tests use. The second
 call would show a dQ accumulator left over from the first one. The file is
 named so pytest collects it last.
 """
@@ -16,7 +18,7 @@ named so pytest collects it last.
 import pytest
 import torch
 
-from tests._parity import GRAD_TOL
+from tests._parity import check_grad, to64
 from workloads import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -46,11 +48,12 @@ def _both(B, H, N, d, causal, seed):
                            scale, int(causal), stream)
     assert st == fa.FA_OK, fa.fa_strerror(st)
     assert fa.fa_get_device_error(stream) == fa.FA_OK
-    for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
-        assert torch.isfinite(g).all().item(), name
-        err = float((g.float() - r.float()).abs().max())
-        bar = GRAD_TOL * float(r.float().abs().max())
-        assert err <= bar, f"{name}: {err:.3e} > {bar:.3e}"
+    assert torch.equal(got[1], ref[1]), "dK differs from fa_bwd"
+    assert torch.equal(got[2], ref[2]), "dV differs from fa_bwd"
+    from oracle import attention_backward
+
+    rq, _, _ = attention_backward(x["q"], x["k"], x["v"], x["do"], scale, causal)
+    check_grad(to64(got[0]), rq, "dQ", f"noalloc B{B} H{H} N{N} d{d} causal={causal}")
 
 
 def test_noalloc_matches_fa_bwd_on_two_calls_in_a_row():
