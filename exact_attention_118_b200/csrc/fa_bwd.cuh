@@ -502,6 +502,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int it = 0; ok && it < n_it; ++it) {
           const int t = it % DOS;
+          // dV(it) reads dO(it): nothing else X waits for implies it landed.
+          if (!(ok = wait_parity(do_full + t, (it / DOS) & 1, abort_flag))) break;
           if (!(ok = wait_parity(p_full, it & 1, abort_flag))) break;
           tc_fence_after();
           issue_acc(t_dv, 0, do_addr + t * L::kTile, it > 0);
@@ -518,6 +520,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       } else if (role == 1) {
         for (int it = 0; ok && it < n_it; ++it) {
           const int s = it % QS;
+          // dS^T(it) implies S^T(it) and so Q(it); the Q wait is explicit anyway.
+          if (!(ok = wait_parity(q_full + s, (it / QS) & 1, abort_flag))) break;
           if (!(ok = wait_parity(ds_full, it & 1, abort_flag))) break;
           tc_fence_after();
           issue_acc(t_dk, t_dp, q_addr + s * L::kTile, it > 0);

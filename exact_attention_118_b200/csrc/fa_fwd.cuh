@@ -88,9 +88,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Every kPolyEvery-th column pair of an unmasked tile takes its exponentials
 // on the FMA pipe (exp2_fma2) instead of the special-function unit; 0: none.
 #ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 4
+#define FA_FWD_POLY_EVERY 8
 #endif
 constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
+// P goes to the PV MMA in two halves (1) or at once (0).
+#ifndef FA_FWD_SPLIT_P
+#define FA_FWD_SPLIT_P 1
+#endif
+constexpr bool kSplitP = FA_FWD_SPLIT_P != 0;
 
 // 2^x for a pair of fp32 values on the FMA pipe, x <= 2^22 (here x <= 8).
 // Cody and Waite's range reduction: n = round(x) by adding and subtracting
@@ -455,9 +460,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             pk[cc] = pack_bf16(pp.x, pp.y);
           }
           tmem_st32(tS + 32 * hh, pk);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(hh ? p_full + t : p_half + t);
+          if (hh == 1 || kSplitP) {
+            tmem_wait_st();
+            tc_fence_before();
+            if (hh == 0 || !kSplitP) mbar_arrive(p_half + t);
+            if (hh == 1) mbar_arrive(p_full + t);
+          }
         };
         if (kPolyEvery > 0 && !masked) {
           half(std::true_type{}, 0);
