@@ -179,21 +179,79 @@ struct Geom {
   int map_heads(int heads) const { return packed() ? heads : B * heads; }
 };
 
-fa_status make_head_map(CUtensorMap* m, const void* base, const Geom& g, int heads, CUtensorMapDataType dt,
-                        int elem_bytes, int inner, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return FA_ERR_CUDA;
-  const cuuint64_t row_bytes = static_cast<cuuint64_t>(inner) * elem_bytes;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(g.rows()),
-                              static_cast<cuuint64_t>(g.map_heads(heads))};
-  const cuuint64_t strides[2] = {g.packed() ? row_bytes * heads : row_bytes,
-                                 g.packed() ? row_bytes : row_bytes * g.N};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+// Encoded tensor maps, cached. A map is a pure function of its encoding
+// arguments (address, sizes, strides, box, type, swizzle), so a cached map
+// equals a fresh encoding of the same arguments whatever happened to the
+// memory in between; the cache only saves the host time of encoding (the
+// calls encode 4 to 9 maps each). Direct-mapped by a hash of the key.
+struct MapKey {
+  const void* base;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  int rank, dtype, swizzle;
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+class MapCache {
+ public:
+  // Encodes (or finds) the map; the result is copied out under the lock.
+  CUresult get(const MapKey& key, CUtensorMap* out) {
+    uint64_t h = 1469598103934665603ull;  // FNV-1a over the key bytes
+    const unsigned char* b = reinterpret_cast<const unsigned char*>(&key);
+    for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ b[i]) * 1099511628211ull;
+    const size_t slot = static_cast<size_t>(h % kSlots);
+    std::lock_guard<std::mutex> lock(mu_);
+    if (valid_[slot] && keys_[slot] == key) {
+      *out = maps_[slot];
+      return CUDA_SUCCESS;
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return CUDA_ERROR_NOT_INITIALIZED;
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(&maps_[slot], static_cast<CUtensorMapDataType>(key.dtype), static_cast<cuuint32_t>(key.rank),
+                     const_cast<void*>(key.base), key.dims, key.strides, key.box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, static_cast<CUtensorMapSwizzle>(key.swizzle),
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    valid_[slot] = (r == CUDA_SUCCESS);
+    if (r != CUDA_SUCCESS) return r;
+    keys_[slot] = key;
+    *out = maps_[slot];
+    return CUDA_SUCCESS;
+  }
+
+ private:
+  static constexpr size_t kSlots = 256;
+  std::mutex mu_;
+  MapKey keys_[kSlots];
+  alignas(64) CUtensorMap maps_[kSlots];
+  bool valid_[kSlots] = {};
+};
+MapCache g_maps;
+
+fa_status encode_map(CUtensorMap* m, const MapKey& key) {
+  if (!encode_fn()) return FA_ERR_CUDA;
+  const CUresult r = g_maps.get(key, m);
   if (r != CUDA_SUCCESS) t_last_cuda_error = kEncodeFailed;
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status make_head_map(CUtensorMap* m, const void* base, const Geom& g, int heads, CUtensorMapDataType dt,
+                        int elem_bytes, int inner, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(inner) * elem_bytes;
+  MapKey key{};
+  key.base = base;
+  key.dims[0] = static_cast<cuuint64_t>(inner);
+  key.dims[1] = static_cast<cuuint64_t>(g.rows());
+  key.dims[2] = static_cast<cuuint64_t>(g.map_heads(heads));
+  key.strides[0] = g.packed() ? row_bytes * heads : row_bytes;
+  key.strides[1] = g.packed() ? row_bytes : row_bytes * g.N;
+  key.box[0] = static_cast<cuuint32_t>(box_inner);
+  key.box[1] = static_cast<cuuint32_t>(box_rows);
+  key.box[2] = 1u;
+  key.rank = 3;
+  key.dtype = static_cast<int>(dt);
+  key.swizzle = static_cast<int>(sw);
+  return encode_map(m, key);
 }
 
 // bf16 tiles of 128 rows x 64 columns (128-byte swizzle).
@@ -299,17 +357,17 @@ fa_status launch_fwd_mask(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 // 2-D fp32 map of a [BH][Np] statistics array (Np >= N, a multiple of 4),
 // dims {N, BH}: a 128-wide row box (one query tile), zero-filled past N.
 fa_status make_stat_map(CUtensorMap* m, const float* base, int N, int Np, int BH) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return FA_ERR_CUDA;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Np) * 4};
-  const cuuint32_t box[2] = {128u, 1u};
-  const cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) t_last_cuda_error = kEncodeFailed;
-  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+  MapKey key{};
+  key.base = base;
+  key.dims[0] = static_cast<cuuint64_t>(N);
+  key.dims[1] = static_cast<cuuint64_t>(BH);
+  key.strides[0] = static_cast<cuuint64_t>(Np) * 4;
+  key.box[0] = 128u;
+  key.box[1] = 1u;
+  key.rank = 2;
+  key.dtype = static_cast<int>(CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  key.swizzle = static_cast<int>(CU_TENSOR_MAP_SWIZZLE_NONE);
+  return encode_map(m, key);
 }
 
 template <int D, int MASK>

@@ -117,6 +117,13 @@ def test_bwd_workload_causal_b1h32_n32768_d128_qk3():
     _sampled_heads(WORKLOADS["causal_b1h32_n32768_d128_qk3"], [(0, 0), (0, 16), (0, 31)])
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_odd_tile_count_n16383(causal):
+    # ceil(16383 / 128) = 128 key and query tiles with a ragged last one, at
+    # the headline length: full oracle comparison of one head.
+    _full_case(1, 1, 16383, 128, causal, seed=16383)
+
+
 def test_bwd_repeat_is_deterministic_up_to_reduction_order():
     # dQ is accumulated with fp32 adds whose order may vary between runs; dK and
     # dV are accumulated in a fixed order on chip and must match bit for bit.
