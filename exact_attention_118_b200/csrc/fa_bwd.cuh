@@ -585,10 +585,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
           const float4 l4 = lse2[c4];
-          pr[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), lam, -l4.x));
-          pr[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), lam, -l4.y));
-          pr[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), lam, -l4.z));
-          pr[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), lam, -l4.w));
+          // Packed f32x2: scale and subtract for two queries per instruction.
+          const float2 lam2 = make_float2(lam, lam);
+          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 0]), __uint_as_float(sv[4 * c4 + 1])), lam2,
+                                   make_float2(-l4.x, -l4.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3])), lam2,
+                                   make_float2(-l4.z, -l4.w));
+          pr[4 * c4 + 0] = ex2(x01.x);
+          pr[4 * c4 + 1] = ex2(x01.y);
+          pr[4 * c4 + 2] = ex2(x23.x);
+          pr[4 * c4 + 3] = ex2(x23.y);
         }
       }
       if (edge) {
@@ -605,6 +611,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
         tmem_st32(tS, pk);  // P^T over this thread's own S^T columns
+      }
+      // dS = (scale P) (dP - D): the scale is applied here, off the dS
+      // phase, which is on the iteration's critical path.
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float2 ps = fmul2(make_float2(pr[2 * c], pr[2 * c + 1]), make_float2(scale, scale));
+        pr[2 * c] = ps.x;
+        pr[2 * c + 1] = ps.y;
       }
       tmem_wait_st();
       tc_fence_before();
@@ -626,12 +640,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c4 = 0; c4 < 8; ++c4) {
           const float4 d4 = dd[8 * h + c4];
           const int q = 32 * h + 4 * c4;
-          const float g0 = pr[q + 0] * (__uint_as_float(dp[4 * c4 + 0]) - d4.x) * scale;
-          const float g1 = pr[q + 1] * (__uint_as_float(dp[4 * c4 + 1]) - d4.y) * scale;
-          const float g2 = pr[q + 2] * (__uint_as_float(dp[4 * c4 + 2]) - d4.z) * scale;
-          const float g3 = pr[q + 3] * (__uint_as_float(dp[4 * c4 + 3]) - d4.w) * scale;
-          pk[2 * c4] = pack_bf16(g0, g1);
-          pk[2 * c4 + 1] = pack_bf16(g2, g3);
+          // Packed f32x2: one sub and one mul per pair of queries.
+          const float2 g01 = fmul2(make_float2(pr[q + 0], pr[q + 1]),
+                                   fsub2(make_float2(__uint_as_float(dp[4 * c4 + 0]), __uint_as_float(dp[4 * c4 + 1])),
+                                         make_float2(d4.x, d4.y)));
+          const float2 g23 = fmul2(make_float2(pr[q + 2], pr[q + 3]),
+                                   fsub2(make_float2(__uint_as_float(dp[4 * c4 + 2]), __uint_as_float(dp[4 * c4 + 3])),
+                                         make_float2(d4.z, d4.w)));
+          pk[2 * c4] = pack_bf16(g01.x, g01.y);
+          pk[2 * c4 + 1] = pack_bf16(g23.x, g23.y);
         }
         // dS^T over dP^T columns this thread has already read.
         tmem_st16(tP + 16 * h, pk);
