@@ -72,18 +72,26 @@ struct FwdLayout {
   static constexpr int kRowBytes = D * ESZ;
   static constexpr int kTile = 128 * kRowBytes;               // one 128-row tile
   static constexpr int kChunks = kRowBytes / 128;             // 128-byte column chunks per row
-  static constexpr int kStages = (kRowBytes == 256) ? 2 : 4;  // K/V ring depth
+  static constexpr int kKStages = (kRowBytes == 256) ? 2 : 4;  // K ring depth
+  static constexpr int kVStages = kKStages;                     // V ring depth
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTile;
   static constexpr int kK = 2 * kTile;
-  static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kBar = kV + kStages * kTile;
+  static constexpr int kV = kK + kKStages * kTile;
+  static constexpr int kBar = kV + kVStages * kTile;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KB alignment
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-constexpr int kFwdThreads = 320;
+// MMA issuing threads: 1, or 2 taking alternate K/V steps (an eleventh
+// warp), so one thread's barrier waits overlap the other's MMA issue.
+#ifndef FA_FWD_ISSUERS
+#define FA_FWD_ISSUERS 2
+#endif
+constexpr int kFwdIssuers = FA_FWD_ISSUERS;
+constexpr int kFwdThreads = kFwdIssuers == 2 ? 352 : 320;
+constexpr int kFwdIssuer2Warp = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Every kPolyEvery-th column pair of an unmasked tile takes its exponentials
 // on the FMA pipe (exp2_fma2) instead of the special-function unit; 0: none.
@@ -128,7 +136,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr int ESZ = FP8 ? 1 : 2;
   using L = FwdLayout<D, ESZ>;
   constexpr int CW = 128 / ESZ;  // elements per 128-byte chunk
-  constexpr int S = L::kStages;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
   constexpr int KCH = L::kChunks;  // 128-byte column chunks per row
 
   extern __shared__ uint8_t smem_raw[];
@@ -137,15 +145,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + S;
-  uint64_t* v_full = k_empty + S;
-  uint64_t* v_empty = v_full + S;
-  uint64_t* s_full = v_empty + S;  // [2]
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;  // [2]
   uint64_t* p_half = s_full + 2;   // [2] P of keys 0-63 in TMEM (and O rescaled)
   uint64_t* p_full = p_half + 2;   // [2] P of keys 64-127 in TMEM
-  uint64_t* o_full = p_full + 2;   // [2]
-  uint64_t* mma_done = o_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* o_full = p_full + 2;   // [2] the tile's last PV done (once per CTA)
+  uint64_t* mma_done = o_full + 2;  // [kFwdIssuers]
+  // [2] with two issuers: turn[i] is arrived on by the other issuer once it
+  // has passed every wait of its step, which makes issuer i's next parity
+  // waits unambiguous (the phase before each is then known to be complete).
+  uint64_t* turn = mma_done + kFwdIssuers;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -198,9 +210,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
@@ -210,7 +224,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(p_full + t, 128);
       mbar_init(o_full + t, 1);
     }
-    mbar_init(mma_done, 1);
+    for (int i = 0; i < kFwdIssuers; ++i) mbar_init(mma_done + i, 1);
+    mbar_init(turn + 0, 1);
+    mbar_init(turn + 1, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -234,25 +250,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * CW, s0 + q0 + 128 * t, hq);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < J; ++j) {
-        const int s = j % S, u = j / S;
-        if (j >= S && !wait_parity(k_empty + s, (u - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(k_full + s, L::kTile);
+        const int sk = j % KS, sv = j % VS;
+        if (j >= KS && !wait_parity(k_empty + sk, (j / KS - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(k_full + sk, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTile + c * 16384, &tm_k, k_full + s, c * CW, s0 + (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kK + sk * L::kTile + c * 16384, &tm_k, k_full + sk, c * CW, s0 + (j0 + j) * 128, bkv);
         k_issued = j + 1;
-        if (j >= S && !wait_parity(v_empty + s, (u - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(v_full + s, L::kTile);
+        if (j >= VS && !wait_parity(v_empty + sv, (j / VS - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(v_full + sv, L::kTile);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTile + c * 16384, &tm_v, v_full + s, c * CW, s0 + (j0 + j) * 128, bkv);
+          tma_load_3d(smem + L::kV + sv * L::kTile + c * 16384, &tm_v, v_full + sv, c * CW, s0 + (j0 + j) * 128, bkv);
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.
       wait_parity_drain(q_full, 0);
-      for (int j = max(0, k_issued - S); j < k_issued; ++j) wait_parity_drain(k_full + j % S, (j / S) & 1);
-      for (int j = max(0, v_issued - S); j < v_issued; ++j) wait_parity_drain(v_full + j % S, (j / S) & 1);
+      for (int j = max(0, k_issued - KS); j < k_issued; ++j) wait_parity_drain(k_full + j % KS, (j / KS) & 1);
+      for (int j = max(0, v_issued - VS); j < v_issued; ++j) wait_parity_drain(v_full + j % VS, (j / VS) & 1);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || (kFwdIssuers == 2 && warp == kFwdIssuer2Warp)) {
     // ---------------------------------------------------------- MMA issuer
+    // Issuer `me` takes K/V steps j = me, me + kFwdIssuers, ...: PV_t(j) of
+    // both tiles, then S_t(j+1). Each tile's PV_t(j) and S_t(j+1) come from
+    // one thread, so S_t(j+1) overwrites P_t(j) only after PV_t(j) read it;
+    // everything that crosses issuers goes through a barrier whose commit
+    // covers all earlier MMAs of the committing thread (s_full_t(j+1) covers
+    // PV_t(j), so PV_t(j+1) and the O rescale before it follow PV_t(j)).
+    const int me = warp == 1 ? 0 : 1;
     if (lane == 0) {
       // S: Q, K both K-major. PV: P from TMEM, V MN-major.
       constexpr uint32_t kIdS = FP8 ? idesc_e4m3(128, 128, 0, 0) : idesc_bf16(128, 128, 0, 0);
@@ -291,9 +314,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       };
 
-      bool ok = wait_parity(q_full, 0, abort_flag) && wait_parity(k_full, 0, abort_flag);
-      if (ok) {
+      bool ok = me == 0 ? (wait_parity(q_full, 0, abort_flag) && wait_parity(k_full, 0, abort_flag)) : true;
+      if (ok && me == 0) {
         tc_fence_after();
+#pragma unroll
         for (int t = 0; t < 2; ++t)
           if (a_t[t] == 0 && b_t[t] > 0) {
             issue_s(t, 0);
@@ -301,12 +325,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         mma_commit(k_empty + 0);
       }
-      for (int j = 0; ok && j < J; ++j) {
-        const int s = j % S;
-        if (!(ok = wait_parity(v_full + s, (j / S) & 1, abort_flag))) break;
+      for (int j = me; ok && j < J; j += kFwdIssuers) {
+        if (kFwdIssuers == 2 && j > 0) {
+          // Issuer 0's k-th step follows issuer 1's (k-1)-th, issuer 1's
+          // k-th follows issuer 0's k-th.
+          const int k = j >> 1;
+          if (!(ok = wait_parity(turn + me, (me == 0 ? k - 1 : k) & 1, abort_flag))) break;
+        }
+        const int s = j % VS;
+        if (!(ok = wait_parity(v_full + s, (j / VS) & 1, abort_flag))) break;
         tc_fence_after();
-        const int jn = j + 1, sn = jn % S;
+        const int jn = j + 1, sn = jn % KS;
         bool k_next = false;
+        // Unrolled, so the per-tile ranges and addresses stay in registers.
+#pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (j >= a_t[t] && j < b_t[t]) {
             if (!(ok = wait_parity(p_half + t, (j - a_t[t]) & 1, abort_flag))) break;
@@ -315,24 +347,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!(ok = wait_parity(p_full + t, (j - a_t[t]) & 1, abort_flag))) break;
             tc_fence_after();
             issue_pv(t, s, true, 1);
-            mma_commit(o_full + t);
+            // The epilogue's signal; within the loop the softmax relies on
+            // s_full instead (a commit covers every earlier MMA of this
+            // thread, so S_t(j+1) done means PV_t(j) done).
+            if (j + 1 == b_t[t]) mma_commit(o_full + t);
           }
           if (t == 1) mma_commit(v_empty + s);
           if (jn >= a_t[t] && jn < b_t[t]) {
             if (!k_next) {
-              if (!(ok = wait_parity(k_full + sn, (jn / S) & 1, abort_flag))) break;
+              if (!(ok = wait_parity(k_full + sn, (jn / KS) & 1, abort_flag))) break;
               tc_fence_after();
               k_next = true;
             }
+            // Every wait of this step is behind us: the other issuer may
+            // start on the next step while this one issues S_1(j+1).
+            if (kFwdIssuers == 2 && t == 1) mbar_arrive(turn + (1 - me));
             issue_s(t, sn);
             mma_commit(s_full + t);
+          } else if (kFwdIssuers == 2 && t == 1) {
+            mbar_arrive(turn + (1 - me));
           }
         }
         if (ok && jn < J) mma_commit(k_empty + sn);
       }
       // Let every MMA this thread issued finish before TMEM is freed.
-      mma_commit(mma_done);
-      wait_parity_drain(mma_done, 0);
+      mma_commit(mma_done + me);
+      wait_parity_drain(mma_done + me, 0);
     }
   } else {
     // ------------------------------------------------------------- softmax
@@ -398,32 +438,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_blk;
         rescale = true;
       }
-      if (j > 0) {
-        // PV_{j-1} finished before S_j (same issuing thread, committed
-        // earlier), so this wait is immediate; it keeps the phase count exact.
-        ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (j - 1) & 1, abort_flag));
-        if (!ok) break;
-        // O is rescaled before the first half of P is handed over: PV_j
-        // accumulates into it from then on.
-        if (__any_sync(0xffffffffu, rescale)) {
-          tc_fence_after();
+      // O is rescaled before the first half of P is handed over: PV_j
+      // accumulates into it from then on. PV_{j-1} is done: S_j's commit,
+      // waited for above, covers every MMA the issuer started before it.
+      auto rescale_o = [&]() {
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c, ov);
-            tmem_wait_ld();
+        for (int c = 0; c < D; c += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c, ov);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + c, ov);
-          }
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tO + c, ov);
         }
-      }
+      };
       // A band can hide a whole tile from some rows: while a row has seen no
       // visible key its m is -inf and its p must come out 0, not NaN.
-      const float neg_m = (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m;
-      const float2 lam2 = make_float2(lam, lam), negm2 = make_float2(neg_m, neg_m);
+      auto neg_max = [&]() { return (MASK == kMaskBand && m == -INFINITY) ? 0.f : -m; };
+      const float2 lam2 = make_float2(lam, lam);
       float2 rs = make_float2(0.f, 0.f);
       if (FP8) {
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) rescale_o();
+        const float neg_m = neg_max();
+        const float2 negm2 = make_float2(neg_m, neg_m);
         // Four e4m3 probabilities per TMEM column: P fills 32 columns.
         uint32_t pk[32];
 #pragma unroll
@@ -445,8 +482,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // exp2 (exp2_fma2), which takes load off the special-function unit;
         // masked tiles keep every exponential on ex2, which gives exactly 0
         // for -inf.
-        auto half = [&](auto use_poly, int hh) {
-          uint32_t pk[32];
+        auto compute = [&](auto use_poly, int hh, float neg_m, uint32_t(&pk)[32], float2& acc) {
+          const float2 negm2 = make_float2(neg_m, neg_m);
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
             const int c = 32 * hh + cc;
@@ -456,9 +493,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               pp = exp2_fma2(x);
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
-            rs = fadd2(rs, pp);
+            acc = fadd2(acc, pp);
             pk[cc] = pack_bf16(pp.x, pp.y);
           }
+        };
+        auto store = [&](int hh, const uint32_t(&pk)[32]) {
           tmem_st32(tS + 32 * hh, pk);
           if (hh == 1 || kSplitP) {
             tmem_wait_st();
@@ -467,20 +506,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (hh == 1) mbar_arrive(p_full + t);
           }
         };
-        if (kPolyEvery > 0 && !masked) {
-          half(std::true_type{}, 0);
-          half(std::true_type{}, 1);
-        } else {
-          half(std::false_type{}, 0);
-          half(std::false_type{}, 1);
-        }
+        auto run = [&](auto use_poly) {
+          uint32_t pk[32];
+          if (j > 0 && __any_sync(0xffffffffu, rescale)) rescale_o();
+          const float neg_m = neg_max();
+          compute(use_poly, 0, neg_m, pk, rs);
+          store(0, pk);
+          compute(use_poly, 1, neg_m, pk, rs);
+          store(1, pk);
+        };
+        if (kPolyEvery > 0 && !masked)
+          run(std::true_type{});
+        else
+          run(std::false_type{});
       }
       l = l * alpha + (rs.x + rs.y);
     }
 
     // ------------------------------------------------------------ epilogue
     if (ok && nt > 0) {
-      ok = __all_sync(0xffffffffu, wait_parity(o_full + t, (nt - 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_parity(o_full + t, 0, abort_flag));
       if (ok) {
         tc_fence_after();
         const float inv_l = (FP8 ? p.o_scale : 1.f) / l;
