@@ -37,6 +37,13 @@
 
 namespace fa {
 
+// The dV MMAs of an iteration wait for its dP^T MMAs to finish (1) or go to
+// the tensor pipe as soon as P is ready (0).
+#ifndef FA_BWD_DP_FIRST
+#define FA_BWD_DP_FIRST 1
+#endif
+constexpr bool kDpFirst = FA_BWD_DP_FIRST != 0;
+
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Row stride (elements) of the per-row statistics in the workspace: N rounded
@@ -505,6 +512,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // dV(it) reads dO(it): nothing else X waits for implies it landed.
           if (!(ok = wait_parity(do_full + t, (it / DOS) & 1, abort_flag))) break;
           if (!(ok = wait_parity(p_full, it & 1, abort_flag))) break;
+          // dP^T(it) is on the critical chain (dP^T -> dS phase -> dK, dQ^T ->
+          // drain -> next dP^T) and dV(it) is not, so dV waits until dP^T(it)
+          // has had the tensor pipe. With one dO stage, dP^T(it+1) needs
+          // dO(it+1), whose load needs dV(it) done, so dp_full cannot be two
+          // phases ahead of this wait.
+          if (kDpFirst && DOS == 1 && !(ok = wait_parity(dp_full, it & 1, abort_flag))) break;
           tc_fence_after();
           issue_acc(t_dv, 0, do_addr + t * L::kTile, it > 0);
           mma_commit(do_empty + t);
