@@ -643,11 +643,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, wait_parity(dp_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // Both halves of this group's dP^T columns in one TMEM round trip.
+      uint32_t dpa[64];
+      tmem_ld32(tP + 0, dpa);
+      tmem_ld32(tP + 32, dpa + 32);
+      tmem_wait_ld();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t dp[32];
-        tmem_ld32(tP + 32 * h, dp);
-        tmem_wait_ld();
+        const uint32_t* dp = dpa + 32 * h;
         uint32_t pk[16];
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
