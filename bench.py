@@ -46,9 +46,9 @@ WORKLOAD = "attention fwd+bwd, B=1 H=16 N=16384 d=128 bf16, non-causal then caus
 # (B=1, H=16, N=16384, d=128): dram__bytes_read.sum + dram__bytes_write.sum
 # from one ncu capture of that very launch shape. None until a capture of the
 # current kernel source exists; a number taken on other source is not used.
-BWD_TRAFFIC = {"bytes": 405780224 + 223552768, "read": 405780224, "write": 223552768,
+BWD_TRAFFIC = {"bytes": 405746944 + 222314752, "read": 405746944, "write": 222314752,
                "shape": "B=1 H=16 N=16384 d=128, non-causal, one launch",
-               "source_sha256": "a48ce42d70bdddaada4345adfce7dfffe046c5b4ef2d0ae2ef04e7e0a8f203b6"}
+               "source_sha256": "c1f89499529faf3d51678bb84beceb1cd2004136299913c67f1f283d6797e2cd"}
 # Dense bf16 tensor-core peak of a B200 as the vendor states it, reported next
 # to the fraction of the measured peak.
 SPEC_BF16_TFLOPS = 2250.0
@@ -535,7 +535,14 @@ def run_next_rows(args):
     def rnd(*shape):
         return torch.randn(*shape, device=dev, generator=g).to(torch.bfloat16)
 
+    # Each row starts after the GPU has idled briefly, so that a row's
+    # figure does not depend on how hot the rows before it left the part
+    # (under the 1 kW power cap the SM clock drops during long busy spells).
+    cooldown_s = 0.25
+
     def timed(fn):
+        torch.cuda.synchronize()
+        time.sleep(cooldown_s)
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
@@ -562,7 +569,7 @@ def run_next_rows(args):
         ff = 4.0 * d * H * vis_pairs
         line = {"row": row, "metric": "attention TFLOPS/s of visible work", "unit": UNIT, "dtype": dtype,
                 "data": "synthetic", "config": config, "steps": args.steps, "warmup": args.warmup,
-                "fwd_ms": ms_f, "fwd_tflops": ff / ms_f / 1e9}
+                "idle_before_each_pass_s": cooldown_s, "fwd_ms": ms_f, "fwd_tflops": ff / ms_f / 1e9}
         line["fwd_frac_of_peak"] = line["fwd_tflops"] / (fwd_peak or peak)
         if ms_b is not None:
             line.update({"bwd_ms": ms_b, "bwd_tflops": 2.5 * ff / ms_b / 1e9,
