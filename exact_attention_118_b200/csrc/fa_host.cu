@@ -300,13 +300,12 @@ unsigned helper_grid(long long threads_needed) {
 // heaviest CTA (about 2 tiles' worth of steps per tile of the longest axis)
 // finishes no later than the group's other CTAs: with `tiles` tiles per unit
 // and work ~ tiles^2 per unit spread over the SMs, that needs a group of at
-// least 2 * SMs / tiles units. Working sets up to twice the L2 gain nothing
-// from grouping (measured), so they keep one group: the global
-// heaviest-first order. Returns the number of groups.
+// least 2 * SMs / tiles units. A working set within one group's budget keeps
+// one group: the global heaviest-first order. Returns the number of groups.
 int sched_groups(long long bytes_per_unit, int units, int tiles) {
-  if (bytes_per_unit * units <= (256ll << 20)) return 1;
+  const long long budget = 64ll << 20;  // streamed operands of one group
+  if (bytes_per_unit * units <= budget) return 1;
   const int sms = sm_count();
-  const long long budget = 64ll << 20;
   long long g_max = bytes_per_unit > 0 ? budget / bytes_per_unit : units;
   if (g_max < 1) g_max = 1;
   long long g_min = tiles > 0 ? (2ll * sms + tiles - 1) / tiles : 1;
