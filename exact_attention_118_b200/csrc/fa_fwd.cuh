@@ -104,6 +104,12 @@ constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 #define FA_FWD_SPLIT_P 1
 #endif
 constexpr bool kSplitP = FA_FWD_SPLIT_P != 0;
+// The FP8 softmax's share on the FMA pipe: every kPolyEvery8-th group of four
+// columns of an unmasked tile (0: none).
+#ifndef FA_FWD_FP8_POLY_EVERY
+#define FA_FWD_FP8_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery8 = FA_FWD_FP8_POLY_EVERY;
 
 // 2^x for a pair of fp32 values on the FMA pipe, x <= 2^22 (here x <= 8).
 // Cody and Waite's range reduction: n = round(x) by adding and subtracting
@@ -461,17 +467,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (j > 0 && __any_sync(0xffffffffu, rescale)) rescale_o();
         const float neg_m = neg_max();
         const float2 negm2 = make_float2(neg_m, neg_m);
-        // Four e4m3 probabilities per TMEM column: P fills 32 columns.
+        // Four e4m3 probabilities per TMEM column: P fills 32 columns. In
+        // unmasked tiles every kPolyEvery8-th column's four exponentials run
+        // on the FMA pipe; e4m3 rounding of P (2^-4 relative) dwarfs the
+        // polynomial's error.
         uint32_t pk[32];
+        auto quads = [&](auto use_poly) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float2 x0 = ffma2(make_float2(s[4 * c], s[4 * c + 1]), lam2, negm2);
-          const float2 x1 = ffma2(make_float2(s[4 * c + 2], s[4 * c + 3]), lam2, negm2);
-          const float2 p01 = make_float2(ex2(x0.x), ex2(x0.y)), p23 = make_float2(ex2(x1.x), ex2(x1.y));
-          rs = fadd2(rs, p01);
-          rs = fadd2(rs, p23);
-          pk[c] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
-        }
+          for (int c = 0; c < 32; ++c) {
+            const float2 x0 = ffma2(make_float2(s[4 * c], s[4 * c + 1]), lam2, negm2);
+            const float2 x1 = ffma2(make_float2(s[4 * c + 2], s[4 * c + 3]), lam2, negm2);
+            float2 p01, p23;
+            if (decltype(use_poly)::value && c % kPolyEvery8 == kPolyEvery8 - 1) {
+              p01 = exp2_fma2(x0);
+              p23 = exp2_fma2(x1);
+            } else {
+              p01 = make_float2(ex2(x0.x), ex2(x0.y));
+              p23 = make_float2(ex2(x1.x), ex2(x1.y));
+            }
+            rs = fadd2(rs, p01);
+            rs = fadd2(rs, p23);
+            pk[c] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);
+          }
+        };
+        if (kPolyEvery8 > 0 && !masked)
+          quads(std::true_type{});
+        else
+          quads(std::false_type{});
         tmem_st32(tS + 0, pk);
         tmem_wait_st();
         tc_fence_before();
