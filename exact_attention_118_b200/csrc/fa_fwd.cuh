@@ -110,6 +110,12 @@ constexpr bool kSplitP = FA_FWD_SPLIT_P != 0;
 #define FA_FWD_FP8_POLY_EVERY 4
 #endif
 constexpr int kPolyEvery8 = FA_FWD_FP8_POLY_EVERY;
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 // 2^x for a pair of fp32 values on the FMA pipe, x <= 2^22 (here x <= 8).
 // Cody and Waite's range reduction: n = round(x) by adding and subtracting
@@ -428,13 +434,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      // Row max with three-input max instructions, in four chains.
+      float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]), mx2 = s[6], mx3 = s[7];
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int c = 8; c < 128; c += 8) {
+        mx0 = fmax3(mx0, s[c], s[c + 1]);
+        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
       }
       const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * lam;
       float alpha = 1.f;
