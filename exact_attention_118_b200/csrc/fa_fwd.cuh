@@ -20,11 +20,11 @@
 //
 // One CTA owns two 128-row query tiles of one (batch, head) and streams the
 // K/V tiles of that head through a shared-memory ring:
-//   warp 0      TMA producer: Q0, Q1 once; K_j, V_j into a KV_STAGES ring.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM, then
-//               O_t += P_t V_j with P_t read from TMEM. The two tiles
-//               alternate so that the tensor core works on one tile while
-//               the other tile's softmax runs.
+//   warp 0      TMA producer: Q0, Q1 once; K_j, V_j into a K/V ring.
+//   warps 1, 10 MMA issuers (one thread each, taking alternate K/V steps):
+//               S_t = Q_t K_j^T into TMEM, then O_t += P_t V_j with P_t read
+//               from TMEM. The two tiles alternate so that the tensor core
+//               works on one tile while the other tile's softmax runs.
 //   warps 2-5   softmax warpgroup of tile 0 (one thread per query row).
 //   warps 6-9   softmax warpgroup of tile 1.
 // TMEM columns (512 allocated): S0/P0 [0,128), S1/P1 [128,256),
