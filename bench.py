@@ -82,9 +82,13 @@ def _bwd_source_sha():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples of one GPU during the timed region."""
+    """nvidia-smi clock/throttle samples of one GPU during the timed region.
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Sampling starts before the region (nvidia-smi takes a while to start) and
+    every sample carries its time stamp; stop() keeps the samples taken
+    between the wall-clock times the region started and ended."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -93,38 +97,46 @@ class ClockSampler:
         self.proc = None
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "20",
                  "-i", gpu_index], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0: float, t1: float):
+        """Summary of the samples stamped within [t0, t1] (wall-clock seconds);
+        all samples, marked as such, if none fall there."""
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except Exception:
             self.proc.kill()
             return None
-        sm, mx, reasons = [], [], set()
+        rows = []
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
             except ValueError:
                 continue
-            for name, val in zip(self.NAMES, f[5:9]):
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside, window = rows, "whole sampling period (none inside the timed region)"
+        if not inside:
+            return None
+        reasons = set()
+        for r in inside:
+            for name, val in zip(self.NAMES, r[3]):
                 if val.lower() == "active":
                     reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
 
 
 # ------------------------------------------------------------ rank helpers
@@ -319,14 +331,16 @@ def run_native(args):
     sampler = ClockSampler(gpu_id)
     time.sleep(0.3)
     start, stop = mk(), mk()
+    t_wall0 = time.time()
     start.record(stream)
     for s in range(args.steps):
         step(evs[s])
     stop.record(stream)
     torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
     barrier()
     torch.cuda.synchronize(dev)
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_wall0, t_wall1)
     check(fa.fa_get_device_error(sp), "timed region")
     ms_total = max_over_ranks(start.elapsed_time(stop), dev)
     ms_per_step, value = aggregate(step_flops, world, ms_total, args.steps)
