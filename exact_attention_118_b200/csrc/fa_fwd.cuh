@@ -96,7 +96,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Every kPolyEvery-th column pair of an unmasked tile takes its exponentials
 // on the FMA pipe (exp2_fma2) instead of the special-function unit; 0: none.
 #ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 8
+#define FA_FWD_POLY_EVERY 6
 #endif
 constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 // P goes to the PV MMA in two halves (1) or at once (0).
