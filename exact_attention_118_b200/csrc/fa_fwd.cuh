@@ -20,7 +20,9 @@
 //
 // One CTA owns two 128-row query tiles of one (batch, head) and streams the
 // K/V tiles of that head through a shared-memory ring:
-//   warp 0      TMA producer: Q0, Q1 once; K_j, V_j into a K/V ring.
+//   warp 0      TMA producer: Q0, K_0, Q1 (each query tile under its own
+//               barrier, so the first S waits for one tile), then K_j, V_j
+//               into a K/V ring.
 //   warps 1, 10 MMA issuers (one thread each, taking alternate K/V steps):
 //               S_t = Q_t K_j^T into TMEM, then O_t += P_t V_j with P_t read
 //               from TMEM. The two tiles alternate so that the tensor core
@@ -110,6 +112,17 @@ constexpr bool kSplitP = FA_FWD_SPLIT_P != 0;
 #define FA_FWD_FP8_POLY_EVERY 4
 #endif
 constexpr int kPolyEvery8 = FA_FWD_FP8_POLY_EVERY;
+// Q_0 and Q_1 under one barrier each, Q_1 loaded after K_0, so the first S
+// waits for one query tile instead of two (1), or both under one barrier (0).
+#ifndef FA_FWD_Q_SPLIT
+#define FA_FWD_Q_SPLIT 1
+#endif
+constexpr bool kQSplit = FA_FWD_Q_SPLIT != 0;
+// The epilogue's TMA stores waited for until their shared-memory source has
+// been read (1) or until the writes are complete (0).
+#ifndef FA_FWD_STORE_WAIT_READ
+#define FA_FWD_STORE_WAIT_READ 1
+#endif
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -155,8 +168,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
+  static_assert(8 * (2 + 2 * KS + 2 * VS + 8 + kFwdIssuers + 2) + 8 <= L::kBytes - L::kBar, "barrier area");
+  uint64_t* q_full = bars + 0;  // [2]: Q_0, Q_1 (only [0] without kQSplit)
+  uint64_t* k_full = bars + 2;
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
@@ -221,7 +235,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int J = max(b_t[0], b_t[1]);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full + 0, 1);
+    mbar_init(q_full + 1, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -256,10 +271,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, 2 * L::kTile);
-      for (int t = 0; t < 2; ++t)
+      auto load_q = [&](int t) {
+        uint64_t* bar = q_full + (kQSplit ? t : 0);
         for (int c = 0; c < KCH; ++c)
-          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, q_full, c * CW, s0 + q0 + 128 * t, hq);
+          tma_load_3d(smem + (t ? L::kQ1 : L::kQ0) + c * 16384, &tm_q, bar, c * CW, s0 + q0 + 128 * t, hq);
+      };
+      if (kQSplit) {
+        mbar_arrive_expect_tx(q_full + 0, L::kTile);
+        mbar_arrive_expect_tx(q_full + 1, L::kTile);
+        load_q(0);
+      } else {
+        mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+        load_q(0);
+        load_q(1);
+      }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < J; ++j) {
         const int sk = j % KS, sv = j % VS;
@@ -268,6 +293,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(smem + L::kK + sk * L::kTile + c * 16384, &tm_k, k_full + sk, c * CW, s0 + (j0 + j) * 128, bkv);
         k_issued = j + 1;
+        if (kQSplit && j == 0) load_q(1);
         if (j >= VS && !wait_parity(v_empty + sv, (j / VS - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + sv, L::kTile);
         for (int c = 0; c < KCH; ++c)
@@ -275,7 +301,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         v_issued = j + 1;
       }
       // Every copy this thread started must land before the CTA exits.
-      wait_parity_drain(q_full, 0);
+      wait_parity_drain(q_full + 0, 0);
+      if (kQSplit) wait_parity_drain(q_full + 1, 0);
       for (int j = max(0, k_issued - KS); j < k_issued; ++j) wait_parity_drain(k_full + j % KS, (j / KS) & 1);
       for (int j = max(0, v_issued - VS); j < v_issued; ++j) wait_parity_drain(v_full + j % VS, (j / VS) & 1);
     }
@@ -332,10 +359,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t)
           if (a_t[t] == 0 && b_t[t] > 0) {
+            if (kQSplit && t == 1) {
+              if (!(ok = wait_parity(q_full + 1, 0, abort_flag))) break;
+              tc_fence_after();
+            }
             issue_s(t, 0);
             mma_commit(s_full + t);
           }
-        mma_commit(k_empty + 0);
+        if (ok) mma_commit(k_empty + 0);
       }
       for (int j = me; ok && j < J; j += kFwdIssuers) {
         if (kFwdIssuers == 2 && j > 0) {
@@ -370,6 +401,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!(ok = wait_parity(k_full + sn, (jn / KS) & 1, abort_flag))) break;
               tc_fence_after();
               k_next = true;
+            }
+            // Query tile 1 joining the stream after the first step (a band).
+            if (kQSplit && t == 1 && jn == a_t[1]) {
+              if (!(ok = wait_parity(q_full + 1, 0, abort_flag))) break;
+              tc_fence_after();
             }
             // Every wait of this step is behind us: the other issuer may
             // start on the next step while this one issues S_1(j+1).
@@ -569,6 +605,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // bf16 O: each warp stages its 32 rows in its part of the tile's Q
           // buffer (free: the tile's last S MMA has read it) with the 128-byte
           // swizzle and writes them with TMA stores, which clip rows past N.
+          // The warp waits only until the stores have read the buffer.
           uint8_t* stg = smem + (t ? L::kQ1 : L::kQ0) + quarter * (32 * D * 2);
           uint8_t* orow = stg + lane * 128;
           const int sw = lane & 7;
@@ -593,7 +630,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) tma_store_3d(&tm_o, stg + c * 4096, 64 * c, s0 + r0, hq);
             bulk_commit_group();
-            bulk_wait_group0();
+            if (FA_FWD_STORE_WAIT_READ)
+              bulk_wait_group_read0();
+            else
+              bulk_wait_group0();
           }
           __syncwarp();
         } else {
