@@ -291,6 +291,8 @@ def run_native(args):
     def run_pass(causal, ev=None, inp=None, out=None):
         o = outs[causal] if out is None else out
         qp, kp, vp, dop = (q, k, v, do) if inp is None else (inp[n].data_ptr() for n in ("q", "k", "v", "do"))
+        if ev is not None:
+            ev[4].record(stream)
         check(fa.fa_fwd(qp, kp, vp, o["o"].data_ptr(), o["lse"].data_ptr(), B, H, N, D, scale, int(causal),
                         fa.FA_BF16, sp), "fa_fwd")
         if ev is not None:
@@ -322,7 +324,7 @@ def run_native(args):
         e.record(stream)  # creates the underlying cudaEvent_t
         return e
 
-    evs = [[[mk() for _ in range(4)] for _ in range(2)] for _ in range(args.steps)]
+    evs = [[[mk() for _ in range(5)] for _ in range(2)] for _ in range(args.steps)]
     gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local] if os.environ.get(
         "CUDA_VISIBLE_DEVICES") else str(local)
     torch.cuda.synchronize(dev)
@@ -356,12 +358,18 @@ def run_native(args):
         bwd_total = [x[0].elapsed_time(x[3]) for x in e]
         main = [x[1].elapsed_time(x[2]) for x in e]
         bwd_main_ms[c] = main
-        per[c] = {"bwd_ms": med(bwd_total), "bwd_main_ms": med(main)}
+        per[c] = {"bwd_ms": med(bwd_total), "bwd_main_ms": med(main),
+                  "fwd_ms": med([x[4].elapsed_time(x[0]) for x in e])}
 
-    # forward alone, timed the same way in its own loop
+    # The forward alone, in a loop of its own that starts after the GPU has
+    # idled briefly (a kernel timed alone, as the burst peak was measured);
+    # the in-step figures above come from the hot step loop.
+    fwd_idle_s = 0.5
     fwd_ms = {}
     for c in (False, True):
         o = outs[c]
+        torch.cuda.synchronize(dev)
+        time.sleep(fwd_idle_s)
         a, b_ = mk(), mk()
         a.record(stream)
         for _ in range(args.steps):
@@ -377,10 +385,15 @@ def run_native(args):
         ff, fb = _flops(c)
         passes[f"fwd_{tag}"] = {"ms": fwd_ms[c], "tflops": ff / fwd_ms[c] / 1e9,
                                 "frac_of_peak": ff / fwd_ms[c] / 1e9 / peak,
-                                "frac_of_spec": ff / fwd_ms[c] / 1e9 / SPEC_BF16_TFLOPS}
+                                "frac_of_spec": ff / fwd_ms[c] / 1e9 / SPEC_BF16_TFLOPS,
+                                "timed": f"alone, {args.steps} launches after {fwd_idle_s} s idle",
+                                "in_step_ms": per[c]["fwd_ms"],
+                                "in_step_tflops": ff / per[c]["fwd_ms"] / 1e9,
+                                "in_step_frac_of_peak": ff / per[c]["fwd_ms"] / 1e9 / peak}
         passes[f"bwd_{tag}"] = {"ms": per[c]["bwd_ms"], "tflops": fb / per[c]["bwd_ms"] / 1e9,
                                 "frac_of_peak": fb / per[c]["bwd_ms"] / 1e9 / peak,
                                 "frac_of_spec": fb / per[c]["bwd_ms"] / 1e9 / SPEC_BF16_TFLOPS,
+                                "timed": "inside the timed step",
                                 "main_kernel_ms": per[c]["bwd_main_ms"]}
 
     # Roofline of the dominant kernel: the main backward kernel, non-causal
