@@ -123,6 +123,26 @@ constexpr bool kQSplit = FA_FWD_Q_SPLIT != 0;
 #ifndef FA_FWD_STORE_WAIT_READ
 #define FA_FWD_STORE_WAIT_READ 1
 #endif
+// TMEM columns of P the softmax packs and stores at a time: 32, 16 or 8.
+// Fewer keep fewer packed values live beside the 128 scores.
+#ifndef FA_FWD_P_ST_COLS
+#define FA_FWD_P_ST_COLS 16
+#endif
+// The warp index read through a shuffle from lane 0 (1), which marks it, and
+// everything derived from it, as the same for all lanes of a warp: the
+// compiler can then keep those values in uniform registers instead of the
+// per-thread ones the 128 scores need.
+#ifndef FA_FWD_UNIFORM_WARP
+#define FA_FWD_UNIFORM_WARP 1
+#endif
+constexpr int kPStCols = FA_FWD_P_ST_COLS;
+static_assert(kPStCols == 32 || kPStCols == 16 || kPStCols == 8, "P store width");
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -186,7 +206,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = FA_FWD_UNIFORM_WARP ? __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0)
+                                      : static_cast<int>(threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
 
   // Causal: heads in sched_groups groups, each small enough that its K/V
@@ -452,24 +473,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       }
       const int kb = (j0 + a_me + j) * 128;
+      // A tile the mask cuts: this row sees keys kb + [lo_m, hi_m).
       bool masked = false;
+      int lo_m = 0, hi_m = 128;
       if (MASK == kMaskBand) {
         const int qs = q0 + 128 * t;
         if (kb + 128 > N || kb + 127 > qs + p.wr || kb < qs + 127 - p.wl) {
           masked = true;
-          const int hi = min(N - kb, qi + p.wr - kb + 1), lo = qi - p.wl - kb;
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= hi || c < lo) s[c] = -INFINITY;
+          hi_m = min(N - kb, qi + p.wr - kb + 1);
+          lo_m = qi - p.wl - kb;
         }
       } else if (kb + 128 > N || (MASK == kMaskCausal && kb + 127 > q0 + 128 * t)) {
         masked = true;
-        int lim = N - kb;
-        if (MASK == kMaskCausal) lim = min(lim, qi - kb + 1);
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+        hi_m = N - kb;
+        if (MASK == kMaskCausal) hi_m = min(hi_m, qi - kb + 1);
       }
+      auto mask_cols = [&](auto c0, auto c1) {
+#pragma unroll
+        for (int c = decltype(c0)::value; c < decltype(c1)::value; ++c)
+          if (c >= hi_m || c < lo_m) s[c] = -INFINITY;
+      };
+      if (masked) mask_cols(std::integral_constant<int, 0>{}, std::integral_constant<int, 128>{});
       // Row max with three-input max instructions, in four chains.
       float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]), mx2 = s[6], mx3 = s[7];
 #pragma unroll
@@ -547,11 +571,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // exp2 (exp2_fma2), which takes load off the special-function unit;
         // masked tiles keep every exponential on ex2, which gives exactly 0
         // for -inf.
-        auto compute = [&](auto use_poly, int hh, float neg_m, uint32_t(&pk)[32], float2& acc) {
+        // Pairs [W q, W q + W) into W packed columns, stored at once.
+        auto part = [&](auto use_poly, int q, float neg_m, float2& acc) {
+          constexpr int W = kPStCols;
           const float2 negm2 = make_float2(neg_m, neg_m);
+          uint32_t pk[W];
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) {
-            const int c = 32 * hh + cc;
+          for (int cc = 0; cc < W; ++cc) {
+            const int c = W * q + cc;
             const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), lam2, negm2);
             float2 pp;
             if (decltype(use_poly)::value && c % kPolyEvery == kPolyEvery - 1)
@@ -561,9 +588,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             acc = fadd2(acc, pp);
             pk[cc] = pack_bf16(pp.x, pp.y);
           }
+          if (W == 32)
+            tmem_st32(tS + W * q, pk);
+          else if (W == 16)
+            tmem_st16(tS + W * q, pk);
+          else
+            tmem_st8(tS + W * q, pk);
         };
-        auto store = [&](int hh, const uint32_t(&pk)[32]) {
-          tmem_st32(tS + 32 * hh, pk);
+        // After each half of P: make the stores visible to the PV MMA, then
+        // hand the half over (both halves at once without kSplitP).
+        auto handover = [&](int hh) {
           if (hh == 1 || kSplitP) {
             tmem_wait_st();
             tc_fence_before();
@@ -572,13 +606,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         };
         auto run = [&](auto use_poly) {
-          uint32_t pk[32];
           if (j > 0 && __any_sync(0xffffffffu, rescale)) rescale_o();
           const float neg_m = neg_max();
-          compute(use_poly, 0, neg_m, pk, rs);
-          store(0, pk);
-          compute(use_poly, 1, neg_m, pk, rs);
-          store(1, pk);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int q = 0; q < 32 / kPStCols; ++q) part(use_poly, hh * (32 / kPStCols) + q, neg_m, rs);
+            handover(hh);
+          }
         };
         if (kPolyEvery > 0 && !masked)
           run(std::true_type{});
