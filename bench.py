@@ -84,8 +84,9 @@ def _bwd_source_sha():
 class ClockSampler:
     """nvidia-smi clock/throttle samples of one GPU during the timed region.
 
-    Sampling starts before the region (nvidia-smi takes a while to start) and
-    every sample carries its time stamp; stop() keeps the samples taken
+    Sampling starts before the region: wait_ready() returns once nvidia-smi
+    has printed its first sample (it can take most of a second to start).
+    Every sample carries its time stamp; stop() keeps the samples taken
     between the wall-clock times the region started and ended."""
 
     QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -95,12 +96,30 @@ class ClockSampler:
 
     def __init__(self, gpu_index: str):
         self.proc = None
+        self.lines = []
+        self.reader = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "20",
                  "-i", gpu_index], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        import threading
+
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def wait_ready(self, timeout: float = 5.0) -> bool:
+        """Wait (at most `timeout` seconds) for the first sample."""
+        t = time.time()
+        while self.proc is not None and not self.lines and time.time() - t < timeout:
+            time.sleep(0.02)
+        return bool(self.lines)
 
     def stop(self, t0: float, t1: float):
         """Summary of the samples stamped within [t0, t1] (wall-clock seconds);
@@ -110,12 +129,13 @@ class ClockSampler:
         time.sleep(0.1)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            return None
+        if self.reader is not None:
+            self.reader.join(timeout=5)
         rows = []
-        for line in out.strip().splitlines():
+        for line in "".join(self.lines).strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 10:
                 continue
@@ -331,7 +351,8 @@ def run_native(args):
     barrier()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(gpu_id)
-    time.sleep(0.3)
+    sampler.wait_ready()
+    time.sleep(0.1)
     start, stop = mk(), mk()
     t_wall0 = time.time()
     start.record(stream)

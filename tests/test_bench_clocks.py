@@ -1,6 +1,6 @@
 """bench.py's clock sampler keeps the nvidia-smi samples stamped inside the
 timed region (host logic only: the nvidia-smi process is replaced by a fake
-that returns canned lines)."""
+and its output by canned lines)."""
 
 import datetime
 import importlib.util
@@ -18,17 +18,14 @@ def _bench():
 
 
 class _FakeProc:
-    def __init__(self, lines):
-        self.lines = lines
-
     def terminate(self):
         pass
 
     def kill(self):
         pass
 
-    def communicate(self, timeout=None):
-        return "\n".join(self.lines), ""
+    def wait(self, timeout=None):
+        return 0
 
 
 def _stamp(t):
@@ -38,7 +35,9 @@ def _stamp(t):
 def _sampler(lines):
     b = _bench()
     s = b.ClockSampler.__new__(b.ClockSampler)
-    s.proc = _FakeProc(lines)
+    s.proc = _FakeProc()
+    s.reader = None
+    s.lines = [line + "\n" for line in lines]
     return s
 
 
@@ -70,3 +69,16 @@ def test_malformed_lines_are_skipped():
              "Not Active", "[N/A], 0, x, y"]
     c = _sampler(lines).stop(t, t + 1)
     assert c["samples"] == 1 and c["sm_mhz"] == 1965.0
+
+
+def test_wait_ready_returns_once_a_sample_arrived():
+    t = time.time()
+    s = _sampler([f"{_stamp(t)}, 0, 1965, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active"])
+    assert s.wait_ready(timeout=0.1) is True
+
+
+def test_wait_ready_gives_up_after_its_timeout():
+    s = _sampler([])
+    t = time.time()
+    assert s.wait_ready(timeout=0.1) is False
+    assert time.time() - t < 1.0
