@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     b_t[t] = (hi > lo) ? hi - j0 : 0;
   }
   const int J = max(b_t[0], b_t[1]);
-  // The early first load where it measured faster (bf16 in and out).
+  // Only the bf16-in, bf16-out instantiations take the early first load: in
+  // the fp32-O and FP8 ones the moved code makes the compiler spill registers.
   constexpr bool kEarly = kEarlyLoad && !OF32 && !FP8;
 
   // K/V head of this query head (grouped-query attention; equal for MHA).
