@@ -142,6 +142,12 @@ constexpr bool kQSplit = FA_FWD_Q_SPLIT != 0;
 #define FA_FWD_EARLY_LOAD 1
 #endif
 constexpr bool kEarlyLoad = FA_FWD_EARLY_LOAD != 0;
+// The commit that releases V_j's ring stage comes after S_1(j+1) is issued
+// (1), so S_1(j+1) is not queued behind it, or between PV_1(j) and S_1(j+1)
+// (0).
+#ifndef FA_FWD_V_RELEASE_LATE
+#define FA_FWD_V_RELEASE_LATE 1
+#endif
 
 constexpr int kPStCols = FA_FWD_P_ST_COLS;
 static_assert(kPStCols == 32 || kPStCols == 16 || kPStCols == 8, "P store width");
@@ -444,7 +450,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // thread, so S_t(j+1) done means PV_t(j) done).
             if (j + 1 == b_t[t]) mma_commit(o_full + t);
           }
-          if (t == 1) mma_commit(v_empty + s);
+          if (t == 1 && !FA_FWD_V_RELEASE_LATE) mma_commit(v_empty + s);
           if (jn >= a_t[t] && jn < b_t[t]) {
             if (!k_next) {
               if (!(ok = wait_parity(k_full + sn, (jn / KS) & 1, abort_flag))) break;
@@ -464,6 +470,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else if (kFwdIssuers == 2 && t == 1) {
             mbar_arrive(turn + (1 - me));
           }
+          if (t == 1 && FA_FWD_V_RELEASE_LATE) mma_commit(v_empty + s);
         }
         if (ok && jn < J) mma_commit(k_empty + sn);
       }
