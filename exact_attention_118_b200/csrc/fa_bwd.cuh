@@ -43,6 +43,12 @@ namespace fa {
 #define FA_BWD_DP_FIRST 1
 #endif
 constexpr bool kDpFirst = FA_BWD_DP_FIRST != 0;
+// Y commits the release of Q(it)'s ring stage after dQ^T(it) is issued (1),
+// so dQ^T, which the dQ drain waits for, is not queued behind the commit; or
+// between dK(it) and dQ^T(it) (0).
+#ifndef FA_BWD_Q_RELEASE_LATE
+#define FA_BWD_Q_RELEASE_LATE 1
+#endif
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -538,9 +544,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!(ok = wait_parity(ds_full, it & 1, abort_flag))) break;
           tc_fence_after();
           issue_acc(t_dk, t_dp, q_addr + s * L::kTile, it > 0);
-          mma_commit(q_empty + s);
+          if (!FA_BWD_Q_RELEASE_LATE) mma_commit(q_empty + s);
           issue_dq();  // over dS^T(it): after dK(it), same thread
           mma_commit(dq_full);
+          if (FA_BWD_Q_RELEASE_LATE) mma_commit(q_empty + s);
         }
       } else {
         if (ok && (ok = wait_parity(do_full, 0, abort_flag))) {
