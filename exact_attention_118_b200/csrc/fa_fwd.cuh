@@ -148,6 +148,11 @@ constexpr bool kEarlyLoad = FA_FWD_EARLY_LOAD != 0;
 #ifndef FA_FWD_V_RELEASE_LATE
 #define FA_FWD_V_RELEASE_LATE 1
 #endif
+// With two issuers: the arrive that lets the other issuer start the next step
+// comes after S_1(j+1) is issued and committed (1), or just before (0).
+#ifndef FA_FWD_TURN_LATE
+#define FA_FWD_TURN_LATE 1
+#endif
 
 constexpr int kPStCols = FA_FWD_P_ST_COLS;
 static_assert(kPStCols == 32 || kPStCols == 16 || kPStCols == 8, "P store width");
@@ -463,10 +468,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tc_fence_after();
             }
             // Every wait of this step is behind us: the other issuer may
-            // start on the next step while this one issues S_1(j+1).
-            if (kFwdIssuers == 2 && t == 1) mbar_arrive(turn + (1 - me));
+            // start on the next step (after S_1(j+1) is queued, with
+            // FA_FWD_TURN_LATE, so that arrive is not on tile 1's chain).
+            if (kFwdIssuers == 2 && t == 1 && !FA_FWD_TURN_LATE) mbar_arrive(turn + (1 - me));
             issue_s(t, sn);
             mma_commit(s_full + t);
+            if (kFwdIssuers == 2 && t == 1 && FA_FWD_TURN_LATE) mbar_arrive(turn + (1 - me));
           } else if (kFwdIssuers == 2 && t == 1) {
             mbar_arrive(turn + (1 - me));
           }
