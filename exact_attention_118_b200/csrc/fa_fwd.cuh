@@ -374,6 +374,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // everything that crosses issuers goes through a barrier whose commit
     // covers all earlier MMAs of the committing thread (s_full_t(j+1) covers
     // PV_t(j), so PV_t(j+1) and the O rescale before it follow PV_t(j)).
+    // Between a P hand-over and the S that follows it the thread issues only
+    // MMAs: the commit that frees V_j's stage and the other issuer's go-ahead
+    // come after S_1(j+1), off each tile's chain P -> PV -> S -> softmax.
     const int me = warp == 1 ? 0 : 1;
     if (lane == 0) {
       // S: Q, K both K-major. PV: P from TMEM, V MN-major.
